@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the Sol-Attn forward (pool + fused routing/attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid] [--beta 0.5]
+    python bench.py --impl reference ...      # the CPU oracle on the host cores
+
+One step = sol_attn_pool + sol_attn_fwd over one batch of the seeded synthetic workload (the
+whole hot path).  Inputs are resident in HBM; L2 is flushed (a 256 MiB write) before every timed
+step and the step is timed on the device with CUDA events.  Rank 0 prints one JSON line.
+
+Metric: dense-equivalent TFLOP/s = 4*B*H*N^2*d / (time of one call); ms per call in
+``ms_per_step``; the fraction of the B200 bf16 tensor peak on the kept (computed) tiles in
+``computed_tile_frac`` and, with the correction flops included, in ``roofline``.
+With N GPUs every rank runs its own replica (no data-path collective); ``value`` sums the work of
+all ranks over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from free_sparse_attention_block_b200 import inputs  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+# DRAM bytes (read + write) per launch of the fused kernel from one ncu capture, keyed by
+# workload and beta, valid only for the kernel source whose sha256 prefix is given.
+NCU_TRAFFIC = {}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("sol_fwd.cu", "sm100.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "free_sparse_attention_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every ~10 ms (read-only)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ flops
+
+def block_lengths(N: int) -> np.ndarray:
+    Nk = (N + 63) // 64
+    n = np.full(Nk, 64, np.int64)
+    n[-1] = N - 64 * (Nk - 1)
+    return n
+
+
+def flop_counts(mask: np.ndarray, N: int, d: int = 128):
+    """Algorithmic flops of one call from the block mask [BH, Nq, Nk] (uint8):
+    kept = 4 d sum_{kept (i,j)} n_i n_j; correction = 4 d sum_{skipped (i,j)} n_i;
+    executed = what the 128x64 MMA tiles of the kernel actually run (union of a tile pair's kept
+    blocks, plus the correction chunks it needs)."""
+    n = block_lengths(N).astype(np.float64)
+    m = mask.astype(bool)
+    kept = 4.0 * d * float(np.einsum("bij,i,j->", m, n, n))
+    corr = 4.0 * d * float(np.einsum("bij,i->", ~m, n))
+    BH, Nq, Nk = m.shape
+    if Nq % 2:
+        m = np.concatenate([m, np.ones((BH, 1, Nk), bool)], axis=1)
+    a, b = m[:, 0::2], m[:, 1::2]
+    union = (a | b).sum()
+    nchunks = (Nk + 63) // 64
+    pad = np.ones((BH, a.shape[1], nchunks * 64 - Nk), bool)
+    both = np.concatenate([a & b, pad], axis=2).reshape(BH, a.shape[1], nchunks, 64)
+    corr_chunks = (~both.all(axis=3)).sum()
+    executed = 4.0 * d * 128 * 64 * float(union + corr_chunks)
+    return dict(kept=kept, corr=corr, executed=executed, density=float(mask.mean()))
+
+
+# ------------------------------------------------------------------------------ oracle arm
+
+def oracle_sample(wl, beta: float, q, k, v, ntiles: int, seed: int = 0):
+    """Time the CPU oracle (as it stands) on ``ntiles`` query tiles; returns (seconds, dense-eq
+    flops of those tiles, description)."""
+    from oracle import sol_ref
+    rng = np.random.default_rng(seed)
+    BH = wl.B * wl.H
+    Nq = wl.nq
+    heads = sorted(set(int(h) for h in rng.integers(0, BH, size=max(1, min(BH, ntiles // 8)))))
+    per = int(math.ceil(ntiles / len(heads)))
+    qh = q.reshape(BH, wl.N, wl.d)
+    kh = k.reshape(BH, wl.N, wl.d)
+    vh = v.reshape(BH, wl.N, wl.d)
+    t0 = time.perf_counter()
+    done = 0
+    for h in heads:
+        tiles = np.sort(rng.choice(Nq, size=min(per, Nq), replace=False)).astype(np.int64)
+        r = sol_ref.forward(qh[h:h + 1], kh[h:h + 1], vh[h:h + 1], beta, units=tiles)
+        assert np.isfinite(r["out"]).all()
+        done += tiles.size
+    dt = time.perf_counter() - t0
+    flops = done * 4.0 * 64 * wl.N * wl.d
+    desc = f"{done} query tiles of 64 rows from {len(heads)} heads of '{wl.name}' (pool+route+attend)"
+    return dt, flops, desc
+
+
+def cores_used() -> int:
+    n = len(os.sched_getaffinity(0))
+    omp = os.environ.get("OMP_NUM_THREADS")
+    return min(n, int(omp)) if omp else n
+
+
+def calibrated_tiles(wl, beta, q, k, v, seconds: float) -> int:
+    """Number of query tiles the oracle processes in about ``seconds`` on this host."""
+    dt, _, _ = oracle_sample(wl, beta, q, k, v, 16, seed=1234)
+    per_tile = max(dt / 16, 1e-4)
+    return int(max(4, min(wl.B * wl.H * wl.nq, round(seconds / per_tile))))
+
+
+def run_reference(args, wl):
+    """The oracle arm: the CPU oracle as it stands, on rank 0 only, each step a bounded sample
+    (sized so that all steps together take about --ref-seconds)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    q, k, v = inputs.gen_workload(wl)
+    tiles = calibrated_tiles(wl, args.beta, q, k, v, args.ref_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        oracle_sample(wl, args.beta, q, k, v, max(2, tiles // 4), seed=99)
+    times, flops = [], []
+    desc = ""
+    for s in range(args.steps):
+        dt, fl, desc = oracle_sample(wl, args.beta, q, k, v, tiles, seed=s)
+        times.append(dt)
+        flops.append(fl)
+    value = sum(flops) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+METRIC = "sparse attn fwd ms/call, dense-equiv TFLOP/s, % B200 BF16 tensor peak"
+UNIT = "TFLOP/s (dense-equivalent)"
+
+
+def config_of(wl, args):
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "grid": list(wl.grid),
+            "beta": args.beta, "tile": 64,
+            "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+    import free_sparse_attention_block_b200 as sol
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sol.load_library()
+
+    q, k, v = inputs.gen_workload(wl)
+    B, H, N, d = q.shape
+    Nq = wl.nq
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+    ws = torch.zeros(sol.sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(tq)
+    dens = torch.empty((B, H, Nq), dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # mask once (outside timing) for the exact algorithmic flop count
+    sol.sol_attn_pool(tk, tv, ws)
+    mask = torch.empty((B, H, Nq, Nq), dtype=torch.uint8, device=dev)
+    st = sol.sol_attn_fwd_debug(tq, tk, tv, args.beta, ws, out, dens, None, mask, None)
+    if st != 0:
+        raise RuntimeError(f"debug forward failed: {sol.STATUS.get(st)}")
+    fc = flop_counts(mask.cpu().numpy().reshape(B * H, Nq, Nq), N, d)
+    del mask
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sol.sol_attn_pool(tk, tv, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        sol.sol_attn_fwd(tq, tk, tv, args.beta, ws, out, dens)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, where = sol.sol_attn_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {sol.STATUS.get(st)} at wait site {where}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    with sampler:
+        for s in range(args.steps):
+            flush.zero_()
+            step(evs[s])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = float(np.mean([a + b for a, b in zip(pool_ms, fwd_ms)]))
+    mean_fwd = float(np.mean(fwd_ms))
+    mean_pool = float(np.mean(pool_ms))
+    st, where = sol.sol_attn_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {sol.STATUS.get(st)} at wait site {where}")
+
+    # max over ranks of the device time
+    t_max = step_ms
+    if world > 1:
+        t = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+
+    dense = wl.dense_flops()
+    value = world * dense / (t_max * 1e-3) / 1e12
+
+    # ---- e2e through the C ABI on pinned host buffers (copies inside the timed region)
+    hq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hout = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
+    hdens = torch.empty((B, H, Nq), dtype=torch.int32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        sol.sol_attn_fwd_host(hq, hk, hv, args.beta, tq, tk, tv, ws, out, hout, dens, hdens)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        sol.sol_attn_fwd_host(hq, hk, hv, args.beta, tq, tk, tv, ws, out, hout, dens, hdens)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert torch.isfinite(hout.float()).all()
+    h2d = 3 * B * H * N * d * 2
+    d2h = B * H * N * d * 2 + B * H * Nq * 4
+
+    # ---- beta sweep (fwd only, same inputs), for the record
+    sweep = []
+    if args.sweep:
+        for beta in wl.betas:
+            m2 = torch.empty((B, H, Nq, Nq), dtype=torch.uint8, device=dev)
+            sol.sol_attn_fwd_debug(tq, tk, tv, beta, ws, out, dens, None, m2, None)
+            fc2 = flop_counts(m2.cpu().numpy().reshape(B * H, Nq, Nq), N, d)
+            del m2
+            ts = []
+            for _ in range(max(3, args.steps // 2)):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                sol.sol_attn_fwd(tq, tk, tv, beta, ws, out, dens)
+                b.record(stream)
+                ts.append((a, b))
+            torch.cuda.synchronize()
+            ms = float(np.mean([a.elapsed_time(b) for a, b in ts]))
+            sweep.append({"beta": beta, "density": round(fc2["density"], 4), "fwd_ms": round(ms, 4),
+                          "dense_equiv_tflops": round(dense / (ms * 1e-3) / 1e12, 1),
+                          "computed_tile_frac": round(fc2["kept"] / (ms * 1e-3) / 1e12 / PEAK_BF16, 4)})
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        nt = calibrated_tiles(wl, args.beta, q, k, v, args.cpu_seconds)
+        dt, fl, desc = oracle_sample(wl, args.beta, q, k, v, nt)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+
+    achieved = (fc["kept"] + fc["corr"]) / (mean_fwd * 1e-3) / 1e12
+    kh = kernel_hash()
+    tr = NCU_TRAFFIC.get((wl.name, args.beta))
+    traffic = tr["bytes"] if tr and tr["kernel"] == kh else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(wl, args) | {"seed": wl.seed},
+        "fwd_ms": mean_fwd, "pool_ms": mean_pool,
+        "pool_gbs": (2 * B * H * N * d * 2 + B * H * Nq * d * 12) / (mean_pool * 1e-3) / 1e9,
+        "density": fc["density"],
+        "computed_tile_frac": fc["kept"] / (mean_fwd * 1e-3) / 1e12 / PEAK_BF16,
+        "computed_tile_frac_sustained": fc["kept"] / (mean_fwd * 1e-3) / 1e12 / PEAK_BF16_SUST,
+        "executed_mma_tflops": fc["executed"] / (mean_fwd * 1e-3) / 1e12,
+        "union_waste": 1.0 - (fc["kept"] + fc["corr"]) / fc["executed"],
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": PEAK_BF16, "unit": "TFLOP/s",
+                     "frac": achieved / PEAK_BF16, "traffic": traffic,
+                     "peak_source": f"bf16_tflops ({PEAK_SRC}; burst)", "kernel": "sol_fwd_kernel",
+                     "algorithmic_flops_per_launch": fc["kept"] + fc["corr"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "sol_attn_fwd_host (pinned host buffers)"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": sampler.summary(),
+        "workspace_bytes": sol.sol_attn_workspace_bytes(B, H, N, d),
+        "kernel_sha": kh,
+    }
+    if sweep:
+        line["sweep"] = sweep
+    print(json.dumps(line), flush=True)
+
+
+PEAKS, PEAK_SRC = load_peaks()
+PEAK_BF16 = float(PEAKS.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+PEAK_BF16_SUST = float(PEAKS.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mid", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--beta", type=float, default=0.5)
+    ap.add_argument("--sweep", action="store_true", help="also time fwd over the workload's beta sweep")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU-baseline sample time")
+    ap.add_argument("--ref-seconds", type=float, default=90.0, help="target total time of the oracle arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    wl = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

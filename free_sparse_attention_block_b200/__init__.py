@@ -1,1 +1,184 @@
-"""Sol-Attn block-sparse attention forward for B200 (sm_100a)."""
+"""Sol-Attn block-sparse attention forward for NVIDIA B200 (sm_100a).
+
+Python binding of the C ABI in include/sol_attn.h.  It only marshals arguments: tensors are
+passed as device pointers with their sizes, and every step of the computation runs in the CUDA
+kernels of ``libsolattn.so``.  There is no CPU or PyTorch fallback; if the library is missing the
+first call raises.
+
+    import torch, free_sparse_attention_block_b200 as sol
+    out, density = sol.forward(q, k, v, beta=0.5)      # q, k, v: bf16 [B, H, N, 128] on cuda
+
+The functions named ``sol_attn_*`` mirror the C entry points one to one.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+__all__ = [
+    "SolError", "load_library", "LIB_PATH", "HEAD_DIM", "TILE", "STATUS",
+    "sol_attn_workspace_bytes", "sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug",
+    "sol_attn_read_status", "sol_attn_fwd_host", "sol_attn_error_string", "forward",
+    "workspace_views",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+HEAD_DIM = 128
+TILE = 64
+STATUS = {0: "SOL_OK", 1: "SOL_ERR_INVALID_ARG", 2: "SOL_ERR_UNSUPPORTED", 3: "SOL_ERR_ALIGNMENT",
+          4: "SOL_ERR_CUDA", 5: "SOL_ERR_TIMEOUT"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SolError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({sol_attn_error_string(status)})")
+
+
+def load_library(path: str | None = None):
+    """Load libsolattn.so (built by ``python -m free_sparse_attention_block_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise ImportError(f"CUDA library {p} is not built; run "
+                              "`python -m free_sparse_attention_block_b200.build`")
+        lib = C.CDLL(p)
+        vp, i, f = C.c_void_p, C.c_int, C.c_float
+        lib.sol_attn_workspace_bytes.argtypes = [i, i, i, i]
+        lib.sol_attn_workspace_bytes.restype = C.c_size_t
+        lib.sol_attn_pool.argtypes = [vp, vp, i, i, i, i, vp, vp]
+        lib.sol_attn_fwd.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp]
+        lib.sol_attn_fwd_debug.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp, i, i, vp]
+        lib.sol_attn_read_status.argtypes = [vp, C.POINTER(C.c_int), vp]
+        lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.sol_attn_error_string.argtypes = [i]
+        lib.sol_attn_error_string.restype = C.c_char_p
+        for name in ("sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug", "sol_attn_read_status",
+                     "sol_attn_fwd_host"):
+            getattr(lib, name).restype = C.c_int
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _shape(t):
+    if t.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    B, H, N, d = t.shape
+    return int(B), int(H), int(N), int(d)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SolError(status, where)
+
+
+def sol_attn_error_string(status: int) -> str:
+    return load_library().sol_attn_error_string(int(status)).decode()
+
+
+def sol_attn_workspace_bytes(B: int, H: int, N: int, d: int = HEAD_DIM) -> int:
+    return int(load_library().sol_attn_workspace_bytes(B, H, N, d))
+
+
+def sol_attn_pool(k, v, workspace, stream=None, check: bool = True) -> int:
+    B, H, N, d = _shape(k)
+    st = load_library().sol_attn_pool(_ptr(k), _ptr(v), B, H, N, d, _ptr(workspace), _stream(stream))
+    if check:
+        _check(st, "sol_attn_pool")
+    return st
+
+
+def sol_attn_fwd(q, k, v, beta: float, workspace, out, density_out=None, stream=None,
+                 check: bool = True) -> int:
+    B, H, N, d = _shape(q)
+    st = load_library().sol_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(beta),
+                                     _ptr(workspace), _ptr(out), _ptr(density_out), _stream(stream))
+    if check:
+        _check(st, "sol_attn_fwd")
+    return st
+
+
+def sol_attn_fwd_debug(q, k, v, beta: float, workspace, out, density_out=None, proxy_out=None,
+                       mask_out=None, stats_out=None, fault_flags: int = 0, timeout_ms: int = 0,
+                       stream=None) -> int:
+    """Returns the status code (it is not raised: tests inspect SOL_ERR_TIMEOUT)."""
+    B, H, N, d = _shape(q)
+    return load_library().sol_attn_fwd_debug(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(beta), _ptr(workspace), _ptr(out),
+        _ptr(density_out), _ptr(proxy_out), _ptr(mask_out), _ptr(stats_out), int(fault_flags),
+        int(timeout_ms), _stream(stream))
+
+
+def sol_attn_read_status(workspace, stream=None):
+    where = C.c_int(0)
+    st = load_library().sol_attn_read_status(_ptr(workspace), C.byref(where), _stream(stream))
+    return st, where.value
+
+
+def sol_attn_fwd_host(h_q, h_k, h_v, beta: float, d_q, d_k, d_v, workspace, d_out, h_out,
+                      d_density=None, h_density=None, stream=None, check: bool = True) -> int:
+    B, H, N, d = _shape(d_q)
+    st = load_library().sol_attn_fwd_host(
+        _ptr(h_q), _ptr(h_k), _ptr(h_v), B, H, N, d, float(beta), _ptr(d_q), _ptr(d_k), _ptr(d_v),
+        _ptr(workspace), _ptr(d_out), _ptr(d_density), _ptr(h_out), _ptr(h_density), _stream(stream))
+    if check:
+        _check(st, "sol_attn_fwd_host")
+    return st
+
+
+def workspace_views(workspace, B: int, H: int, N: int):
+    """Views of the pooled arrays inside a workspace tensor (uint8, device): (kbar32, vbar32,
+    kbar16, vbar16) shaped [B, H, Nk, 128]; the layout mirrors the C library's."""
+    import torch
+    Nk = (N + TILE - 1) // TILE
+    n = B * H * Nk * HEAD_DIM
+    up = lambda x: (x + 255) & ~255
+    o_k32 = 256
+    o_v32 = up(o_k32 + 4 * n)
+    o_k16 = up(o_v32 + 4 * n)
+    o_v16 = up(o_k16 + 2 * n)
+    shp = (B, H, Nk, HEAD_DIM)
+    k32 = workspace[o_k32:o_k32 + 4 * n].view(torch.float32).view(shp)
+    v32 = workspace[o_v32:o_v32 + 4 * n].view(torch.float32).view(shp)
+    k16 = workspace[o_k16:o_k16 + 2 * n].view(torch.bfloat16).view(shp)
+    v16 = workspace[o_v16:o_v16 + 2 * n].view(torch.bfloat16).view(shp)
+    return k32, v32, k16, v16
+
+
+def forward(q, k, v, beta: float, stream=None):
+    """Pool + fused forward on device tensors.  Allocates the workspace, output and density with
+    torch (the library itself allocates nothing).  Returns (out bf16 [B,H,N,d], density int32
+    [B,H,Nq])."""
+    import torch
+    B, H, N, d = _shape(q)
+    ws = torch.empty(sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q)
+    dens = torch.empty((B, H, (N + TILE - 1) // TILE), dtype=torch.int32, device=q.device)
+    sol_attn_pool(k, v, ws, stream)
+    sol_attn_fwd(q, k, v, beta, ws, out, dens, stream)
+    return out, dens

@@ -1,0 +1,47 @@
+// Internal launch interface between the C-ABI host code and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace sol {
+
+constexpr int kHeadDim = 128;        // d
+constexpr int kTile = 64;            // query tile / key block length T
+constexpr int kMaxBlocks = 8192;     // Nk limit: two proxy rows must fit the 64 KB K/V ring
+constexpr size_t kHeaderBytes = 256; // workspace header (status words)
+
+// Device status words (first bytes of the workspace header).
+struct DeviceStatus {
+    int code;   // 0 = ok, otherwise a sol_status value
+    int where;  // which wait gave up (see WaitSite in sol_fwd.cu)
+};
+
+// Workspace carve-up, all offsets in bytes from the workspace base.
+struct WorkspaceLayout {
+    size_t kbar32, vbar32, kbar16, vbar16, total;
+};
+WorkspaceLayout workspace_layout(long long BH, long long Nk);
+
+cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, float *kbar32,
+                           float *vbar32, void *kbar16, void *vbar16, cudaStream_t stream);
+
+struct FwdLaunch {
+    const CUtensorMap *tm_q, *tm_k, *tm_v, *tm_kb, *tm_vb;
+    int BH, N, Nk, Nq;
+    float beta;
+    const float *kbar32;
+    void *out;
+    int32_t *density;
+    DeviceStatus *status;
+    float *dbg_proxy;
+    uint8_t *dbg_mask;
+    float *dbg_stats;
+    int fault_flags;
+    unsigned long long timeout_ns;
+};
+cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream);
+
+}  // namespace sol

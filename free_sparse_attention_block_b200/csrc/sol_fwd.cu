@@ -1,0 +1,726 @@
+// Fused Sol-Attn forward for sm_100a: routing, exact block-sparse attention and the pooled
+// correction of skipped blocks in one online-softmax pass.
+//
+// Source: "Sol-Attn: Accelerating Video Generation Inference via On-the-Fly Attention
+// Sparsification" (Li et al., 2026): the routing paragraphs (per-query proxy scores against key
+// blocks, their mean mu and standard deviation sigma, keep a block iff its score >= mu +
+// beta*sigma) and the paragraph on the fused operator (routing is not a separate pass before the
+// sparse attention, and skipped blocks are approximated rather than dropped).
+//
+// One CTA owns one 128-row MMA tile = two adjacent 64-row routing tiles (A: rows 0-63, B: rows
+// 64-127) of one head.  Two CTAs fit on an SM (about 104 KB of shared memory and 256 TMEM
+// columns each), so one CTA's routing and softmax overlap the other's tensor-core work.
+//
+//  1. Routing (all 6 warps).  TMA brings the Q tile into shared memory; q_bar of each routing
+//     tile is summed from it in float32; every warp computes proxy scores
+//     S_j = (q_bar . k_bar_j) / sqrt(d) for its key blocks (float32 k_bar_j read from the pooled
+//     workspace) into two shared-memory rows that alias the K/V ring; mu and sigma are reduced in
+//     double with warp shuffles; blocks with S_j >= tau become bit masks (tile A, tile B, union).
+//     The proxy rows never reach global memory (except through the debug outputs).
+//  2. Pipeline.  Work items are first the 64-wide chunks of pooled blocks that still hold a
+//     skipped block (the correction), then every block kept by tile A or tile B (the exact part).
+//     Warp 4 (one lane) streams the item's 64x128 K and V tiles by TMA into a 2-stage ring.
+//     Warp 5 (one lane) issues S = Q K^T (M=128, N=64, K=128) into TMEM, and once the softmax has
+//     written P, O += P V (M=128, N=128, K=64) with P read straight from TMEM.
+//     Warps 0-3 (one thread per row) load S from TMEM, apply the per-row routing decision
+//     (a row of tile A ignores blocks only tile B kept, and vice versa; a correction column is
+//     -inf if the row's tile kept that block, else its logit gets + log2(n_j)), keep a running
+//     max (rescaling O in TMEM only when the max grows by more than 2^8), and store P as bf16
+//     over the first 32 columns of the same TMEM buffer.
+//  3. Epilogue: O / l rounded to bf16 and written to global memory.
+//
+// Every mbarrier wait is bounded (globaltimer): on expiry the CTA records SOL_ERR_TIMEOUT and the
+// wait site in the workspace status words, sets a shared abort flag, lets in-flight TMA copies
+// and MMAs land, frees its TMEM and exits.
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace sol {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kNumWarps = 6;
+constexpr int kWarpTma = 4;
+constexpr int kWarpMma = 5;
+constexpr int kBM = 128;
+
+constexpr uint32_t kQHalfBytes = kBM * 64 * 2;         // 128 rows x 64 channels, bf16
+constexpr uint32_t kQBytes = 2 * kQHalfBytes;
+constexpr uint32_t kKVHalfBytes = kTile * 64 * 2;      // 64 rows x 64 channels, bf16
+constexpr uint32_t kKVTileBytes = 2 * kKVHalfBytes;
+constexpr int kStages = 2;
+
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemO = 128;                       // O accumulator: columns 128..255
+__device__ __forceinline__ uint32_t tmem_s_col(int b) { return b ? 64u : 0u; }
+
+constexpr float kRescaleLog2 = 8.0f;                   // rescale O only if the max grows > 2^8
+
+constexpr int kMaskWords = kMaxBlocks / 32;
+constexpr int kChunkWords = (kMaxBlocks / 64 + 31) / 32;
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kQBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kKVTileBytes;
+constexpr uint32_t kOffMisc = kOffV + kStages * kKVTileBytes;
+constexpr uint32_t kOffRowA = kOffK;                   // proxy rows alias the K/V ring
+constexpr uint32_t kOffRowB = kOffK + kMaxBlocks * 4;
+static_assert(kOffRowB + kMaxBlocks * 4 <= kOffMisc, "proxy rows must fit in the K/V ring");
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, 64, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, 128, true);
+
+enum WaitSite : int {
+    kSiteQ = 1, kSiteProdK = 2, kSiteProdV = 3, kSiteMmaK = 4, kSiteMmaP = 5, kSiteMmaV = 6,
+    kSiteSoftS = 7, kSiteSoftO = 8, kSiteEpilogue = 9, kSiteFault = 10, kSiteDrain = 11,
+    kSiteProdDrain = 12
+};
+
+struct Misc {
+    double red[2][kNumWarps];
+    double mu[2], sigma[2], tau[2];
+    uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+    uint64_t s_full[2], p_full[2], o_done, drain, never;
+    uint32_t mask_a[kMaskWords];
+    uint32_t mask_b[kMaskWords];
+    uint32_t mask_u[kMaskWords];
+    uint32_t need[kChunkWords];
+    float qbar[2][kHeadDim];
+    uint32_t tmem_base;
+    int abort_flag;
+    int count_a, count_b;
+};
+
+constexpr uint32_t kSmemBytes = kOffMisc + sizeof(Misc) + 1024;   // + alignment slack
+
+struct Params {
+    int BH, N, Nk, Nq, npairs, nchunks;
+    float beta;
+    float scale;           // (float)(1/sqrt(d)) for the proxy
+    float scale_log2;      // log2(e)/sqrt(d) for the softmax
+    float last_bias_log2;  // log2(n_last) for the last (possibly partial) block
+    const float *kbar32;
+    __nv_bfloat16 *out;
+    int32_t *density;
+    DeviceStatus *status;
+    float *dbg_proxy;
+    uint8_t *dbg_mask;
+    float *dbg_stats;
+    int fault_flags;
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ int volatile_load(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
+
+// Bounded wait on an mbarrier phase.  honor_abort=false is used while draining in-flight copies.
+__device__ bool wait_bar(uint64_t *bar, uint32_t parity, Misc &m, const Params &p, int site,
+                         bool honor_abort = true)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (honor_abort && volatile_load(&m.abort_flag)) return false;
+            if (globaltimer_ns() - t0 > p.timeout_ns) {
+                *reinterpret_cast<volatile int *>(&m.abort_flag) = 1;
+                if (atomicCAS(&p.status->code, 0, 5) == 0) atomicExch(&p.status->where, site);
+                return false;
+            }
+        }
+    }
+}
+
+// Smallest set bit index >= from (and < limit) in a bit array, or -1.
+__device__ __forceinline__ int next_bit(const uint32_t *bits, int from, int limit)
+{
+    if (from >= limit) return -1;
+    int w = from >> 5;
+    uint32_t word = bits[w] & (0xFFFFFFFFu << (from & 31));
+    const int nw = (limit + 31) >> 5;
+    for (;;) {
+        if (word) {
+            const int r = (w << 5) + __ffs(word) - 1;
+            return r < limit ? r : -1;
+        }
+        if (++w >= nw) return -1;
+        word = bits[w];
+    }
+}
+
+// The work-item sequence every role walks identically: correction chunks, then kept blocks.
+struct Walker {
+    int phase = 0;   // 0: correction chunks, 1: kept blocks, 2: done
+    int idx = -1;
+    __device__ __forceinline__ bool next(const Misc &m, const Params &p)
+    {
+        if (phase == 0) {
+            const int c = next_bit(m.need, idx + 1, p.nchunks);
+            if (c >= 0) { idx = c; return true; }
+            phase = 1;
+            idx = -1;
+        }
+        if (phase == 1) {
+            const int j = next_bit(m.mask_u, idx + 1, p.Nk);
+            if (j >= 0) { idx = j; return true; }
+            phase = 2;
+        }
+        return false;
+    }
+};
+
+__device__ __forceinline__ float bf16_at(const uint8_t *p)
+{
+    return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(p)) << 16);
+}
+
+// ----------------------------------------------------------------------------- roles
+
+__device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                              const CUtensorMap *tm_kb, const CUtensorMap *tm_vb, uint8_t *smem,
+                              Misc &m, const Params &p, int bh)
+{
+    int issued_k[kStages], issued_v[kStages];
+    for (int s = 0; s < kStages; ++s) issued_k[s] = issued_v[s] = -1;
+    Walker w;
+    int it = 0;
+    while (w.next(m, p)) {
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const bool corr = w.phase == 0;
+        const CUtensorMap *mk = corr ? tm_kb : tm_k;
+        const CUtensorMap *mv = corr ? tm_vb : tm_v;
+        const int row = w.idx * kTile;
+        uint8_t *kdst = smem + kOffK + s * kKVTileBytes;
+        uint8_t *vdst = smem + kOffV + s * kKVTileBytes;
+        if (!wait_bar(&m.k_empty[s], ph ^ 1u, m, p, kSiteProdK)) break;
+        mbar_arrive_expect_tx(&m.k_full[s], kKVTileBytes);
+        tma_load_3d(kdst, mk, &m.k_full[s], 0, row, bh);
+        tma_load_3d(kdst + kKVHalfBytes, mk, &m.k_full[s], 64, row, bh);
+        issued_k[s] = it;
+        if (!wait_bar(&m.v_empty[s], ph ^ 1u, m, p, kSiteProdV)) break;
+        mbar_arrive_expect_tx(&m.v_full[s], kKVTileBytes);
+        tma_load_3d(vdst, mv, &m.v_full[s], 0, row, bh);
+        tma_load_3d(vdst + kKVHalfBytes, mv, &m.v_full[s], 64, row, bh);
+        issued_v[s] = it;
+        ++it;
+    }
+    // No TMA write may still be in flight when the CTA exits.
+    for (int s = 0; s < kStages; ++s) {
+        if (issued_k[s] >= 0) wait_bar(&m.k_full[s], (issued_k[s] >> 1) & 1, m, p, kSiteProdDrain, false);
+        if (issued_v[s] >= 0) wait_bar(&m.v_full[s], (issued_v[s] >> 1) & 1, m, p, kSiteProdDrain, false);
+    }
+}
+
+__device__ __forceinline__ bool issue_pv(int t, uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
+{
+    const int b = t & 1, s = t & 1;
+    const uint32_t ph = (t >> 1) & 1;
+    if (!wait_bar(&m.p_full[b], ph, m, p, kSiteMmaP)) return false;
+    if (!wait_bar(&m.v_full[s], ph, m, p, kSiteMmaV)) return false;
+    tc_fence_after();
+    const uint32_t v_base = smem_u32(smem + kOffV + s * kKVTileBytes);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        // B = V tile, MN-major: 64 channels contiguous per key row (128 B, swizzled), next 8 keys
+        // at +1024 B (SBO), channels 64..127 at +8192 B (LBO); 16 keys per MMA -> +2048 B.
+        const uint64_t bdesc = desc_sw128(v_base + kk * 2048, kKVHalfBytes, 1024);
+        mma_ts(tmem + kTmemO, tmem + tmem_s_col(b) + kk * 8, bdesc, kIdescPV,
+               (t > 0 || kk > 0) ? 1u : 0u);
+    }
+    mma_commit(&m.v_empty[s]);
+    mma_commit(&m.o_done);
+    return true;
+}
+
+__device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
+{
+    bool ok = true;
+    if (p.fault_flags & 1) ok = wait_bar(&m.never, 0, m, p, kSiteFault);
+    if (ok) ok = wait_bar(&m.q_full, 0, m, p, kSiteQ);
+    if (ok) {
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(smem + kOffQ);
+        Walker w;
+        int it = 0;
+        while (ok && w.next(m, p)) {
+            const int s = it & 1, b = it & 1;
+            if (!wait_bar(&m.k_full[s], (it >> 1) & 1, m, p, kSiteMmaK)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(smem + kOffK + s * kKVTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                // A = Q (128 x 128), B = K tile (64 x 128), both K-major 128B-swizzled with 8-row
+                // groups 1024 B apart; channels 64..127 live in the second half buffer and a
+                // 16-channel step advances the start address by 32 B inside the swizzle atom.
+                const uint32_t half = kk >> 2, koff = (kk & 3) * 32;
+                const uint64_t adesc = desc_sw128(q_base + half * kQHalfBytes + koff, 16, 1024);
+                const uint64_t bdesc = desc_sw128(k_base + half * kKVHalfBytes + koff, 16, 1024);
+                mma_ss(tmem + tmem_s_col(b), adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&m.k_empty[s]);
+            mma_commit(&m.s_full[b]);
+            if (it > 0 && !issue_pv(it - 1, tmem, smem, m, p)) { ok = false; break; }
+            ++it;
+        }
+        if (ok && it > 0) issue_pv(it - 1, tmem, smem, m, p);
+    }
+    // Every MMA issued so far must finish before TMEM is freed.
+    mma_commit(&m.drain);
+    wait_bar(&m.drain, 0, m, p, kSiteDrain, false);
+}
+
+__device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, int row0)
+{
+    const int row = threadIdx.x;                       // 0..127 == TMEM lane
+    const int warp = row >> 5;
+    const bool in_b = row >= 64;
+    const uint32_t *mymask = in_b ? m.mask_b : m.mask_a;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_used = -INFINITY, l = 0.0f;
+    Walker w;
+    int it = 0;
+    bool ok = true;
+    while (w.next(m, p)) {
+        const int b = it & 1;
+        ok = wait_bar(&m.s_full[b], (it >> 1) & 1, m, p, kSiteSoftS);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_base + tmem_s_col(b);
+        uint32_t pk[32];
+        bool rescale = false;
+        float factor = 1.0f;
+        const bool participate =
+            w.phase == 0 || ((mymask[w.idx >> 5] >> (w.idx & 31)) & 1u);   // warp-uniform
+        if (participate) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(s_addr, r0);
+            tmem_ld32(s_addr + 32, r1);
+            tmem_wait_ld();
+            float x[64];
+            if (w.phase == 0) {
+                const int c = w.idx;
+                const uint64_t sel = static_cast<uint64_t>(mymask[2 * c]) |
+                                     (static_cast<uint64_t>(mymask[2 * c + 1]) << 32);
+                const int j0 = c * 64;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const int j = j0 + i;
+                    const float s = __uint_as_float(i < 32 ? r0[i] : r1[i - 32]);
+                    const float bias = (j == p.Nk - 1) ? p.last_bias_log2 : 6.0f;
+                    const bool use = (j < p.Nk) && !((sel >> i) & 1ull);
+                    x[i] = use ? fmaf(s, p.scale_log2, bias) : -INFINITY;
+                }
+            } else {
+                const int t0 = w.idx * kTile;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const float s = __uint_as_float(i < 32 ? r0[i] : r1[i - 32]);
+                    x[i] = (t0 + i < p.N) ? s * p.scale_log2 : -INFINITY;
+                }
+            }
+            float mx = x[0];
+#pragma unroll
+            for (int i = 1; i < 64; ++i) mx = fmaxf(mx, x[i]);
+            const float m_new = fmaxf(m_used, mx);
+            if (m_new > m_used + kRescaleLog2) {
+                factor = ex2_approx(m_used - m_new);
+                rescale = m_used != -INFINITY;
+                m_used = m_new;
+            }
+            const float mref = m_used == -INFINITY ? 0.0f : m_used;
+            float sum = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float e0 = ex2_approx(x[2 * i] - mref);
+                const float e1 = ex2_approx(x[2 * i + 1] - mref);
+                sum += e0 + e1;
+                pk[i] = pack_bf16x2(e0, e1);
+            }
+            l = l * factor + sum;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        }
+        if (__any_sync(0xFFFFFFFFu, rescale) && it > 0) {
+            ok = wait_bar(&m.o_done, (it - 1) & 1, m, p, kSiteSoftO);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const float f = rescale ? factor : 1.0f;
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t o[32];
+                const uint32_t oaddr = tmem + lane_base + kTmemO + ch * 32;
+                tmem_ld32(oaddr, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                tmem_st32(oaddr, o);
+            }
+        }
+        tmem_st32(s_addr, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&m.p_full[b]);
+        ++it;
+    }
+    if (!ok || it == 0) return;
+    ok = wait_bar(&m.o_done, (it - 1) & 1, m, p, kSiteEpilogue);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (!ok) return;
+    tc_fence_after();
+    const int grow = row0 + row;
+    const bool store = grow < p.N;
+    const float inv_l = 1.0f / l;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + (store ? grow : 0)) * kHeadDim);
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + kTmemO + ch * 32, o);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * inv_l, __uint_as_float(o[8 * q4 + 1]) * inv_l);
+                v.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv_l, __uint_as_float(o[8 * q4 + 3]) * inv_l);
+                v.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv_l, __uint_as_float(o[8 * q4 + 5]) * inv_l);
+                v.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv_l, __uint_as_float(o[8 * q4 + 7]) * inv_l);
+                dst[ch * 4 + q4] = v;
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- kernel
+
+__global__ void __launch_bounds__(kThreads, 2)
+sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
+               const __grid_constant__ CUtensorMap tm_vb, const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Misc &m = *reinterpret_cast<Misc *>(smem + kOffMisc);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pair = blockIdx.x % p.npairs;
+    const int bh = blockIdx.x / p.npairs;
+    const int tile_a = 2 * pair, tile_b = 2 * pair + 1;
+    const bool has_b = tile_b < p.Nq;
+    const int row0 = tile_a * kTile;
+    const int n_a = min(kTile, p.N - row0);
+    const int n_b = has_b ? min(kTile, p.N - row0 - kTile) : 0;
+    const int Nk = p.Nk;
+
+    if (tid == 0) {
+        mbar_init(&m.q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&m.k_full[s], 1);
+            mbar_init(&m.k_empty[s], 1);
+            mbar_init(&m.v_full[s], 1);
+            mbar_init(&m.v_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&m.s_full[b], 1);
+            mbar_init(&m.p_full[b], 128);
+        }
+        mbar_init(&m.o_done, 1);
+        mbar_init(&m.drain, 1);
+        mbar_init(&m.never, 1);
+        m.abort_flag = 0;
+        m.count_a = 0;
+        m.count_b = 0;
+        fence_mbar_init();
+    }
+    for (int i = tid; i < kMaskWords; i += kThreads) {
+        m.mask_a[i] = 0u;
+        m.mask_b[i] = 0u;
+        m.mask_u[i] = 0u;
+    }
+    if (tid < kChunkWords) m.need[tid] = 0u;
+    if (warp == kWarpTma && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_kb);
+        tma_prefetch_desc(&tm_vb);
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(&m.tmem_base, kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = m.tmem_base;
+
+    if (warp == kWarpTma && lane == 0) {
+        mbar_arrive_expect_tx(&m.q_full, kQBytes);
+        tma_load_3d(smem + kOffQ, &tm_q, &m.q_full, 0, row0, bh);
+        tma_load_3d(smem + kOffQ + kQHalfBytes, &tm_q, &m.q_full, 64, row0, bh);
+    }
+
+    // ---------------- routing 1: q_bar of both routing tiles (float32, ascending rows)
+    if (tid < kHeadDim) {
+        if (wait_bar(&m.q_full, 0, m, p, kSiteQ)) {
+            const int c = tid, half = c >> 6, cc = c & 63, chunk = cc >> 3, within = cc & 7;
+            const uint8_t *qh = smem + kOffQ + half * kQHalfBytes + within * 2;
+            float sa = 0.0f, sb = 0.0f;
+            for (int r = 0; r < n_a; ++r) sa += bf16_at(qh + r * 128 + ((chunk ^ (r & 7)) << 4));
+            for (int r = 0; r < n_b; ++r) {
+                const int rr = kTile + r;
+                sb += bf16_at(qh + rr * 128 + ((chunk ^ (rr & 7)) << 4));
+            }
+            m.qbar[0][c] = __fmul_rn(sa, __frcp_rn(static_cast<float>(n_a)));
+            m.qbar[1][c] = has_b ? __fmul_rn(sb, __frcp_rn(static_cast<float>(n_b))) : 0.0f;
+        }
+    }
+    __syncthreads();
+
+    // ---------------- routing 2: proxy rows S_j = (q_bar . k_bar_j) * (1/sqrt d)
+    float *row_a = reinterpret_cast<float *>(smem + kOffRowA);
+    float *row_b = reinterpret_cast<float *>(smem + kOffRowB);
+    const size_t unit_a = static_cast<size_t>(bh) * p.Nq + tile_a;
+    {
+        const float4 qa = reinterpret_cast<const float4 *>(m.qbar[0])[lane];
+        const float4 qb = reinterpret_cast<const float4 *>(m.qbar[1])[lane];
+        const float4 *kb = reinterpret_cast<const float4 *>(p.kbar32 + static_cast<size_t>(bh) * Nk * kHeadDim) + lane;
+        double sum_a = 0.0, sum_b = 0.0;
+        int j = warp;
+        for (; j + 3 * kNumWarps < Nk; j += 4 * kNumWarps) {
+            float4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = __ldg(kb + static_cast<size_t>(j + u * kNumWarps) * 32);
+            float a[4], b[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                a[u] = fmaf(qa.w, x[u].w, fmaf(qa.z, x[u].z, fmaf(qa.y, x[u].y, qa.x * x[u].x)));
+                b[u] = fmaf(qb.w, x[u].w, fmaf(qb.z, x[u].z, fmaf(qb.y, x[u].y, qb.x * x[u].x)));
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    a[u] += __shfl_xor_sync(0xFFFFFFFFu, a[u], o);
+                    b[u] += __shfl_xor_sync(0xFFFFFFFFu, b[u], o);
+                }
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int jj = j + u * kNumWarps;
+                    const float sa = a[u] * p.scale, sb = b[u] * p.scale;
+                    row_a[jj] = sa;
+                    row_b[jj] = sb;
+                    sum_a += sa;
+                    sum_b += sb;
+                }
+            }
+        }
+        for (; j < Nk; j += kNumWarps) {
+            const float4 x = __ldg(kb + static_cast<size_t>(j) * 32);
+            float a = fmaf(qa.w, x.w, fmaf(qa.z, x.z, fmaf(qa.y, x.y, qa.x * x.x)));
+            float b = fmaf(qb.w, x.w, fmaf(qb.z, x.z, fmaf(qb.y, x.y, qb.x * x.x)));
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+                b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+            }
+            if (lane == 0) {
+                const float sa = a * p.scale, sb = b * p.scale;
+                row_a[j] = sa;
+                row_b[j] = sb;
+                sum_a += sa;
+                sum_b += sb;
+            }
+        }
+        if (lane == 0) {
+            m.red[0][warp] = sum_a;
+            m.red[1][warp] = sum_b;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double sa = 0.0, sb = 0.0;
+        for (int w = 0; w < kNumWarps; ++w) { sa += m.red[0][w]; sb += m.red[1][w]; }
+        m.mu[0] = sa / Nk;
+        m.mu[1] = sb / Nk;
+    }
+    __syncthreads();
+    // ---------------- routing 3: sigma (two-pass, double)
+    {
+        const double mu_a = m.mu[0], mu_b = m.mu[1];
+        double ss_a = 0.0, ss_b = 0.0;
+        for (int j = tid; j < Nk; j += kThreads) {
+            const double da = static_cast<double>(row_a[j]) - mu_a;
+            const double db = static_cast<double>(row_b[j]) - mu_b;
+            ss_a += da * da;
+            ss_b += db * db;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            ss_a += __shfl_xor_sync(0xFFFFFFFFu, ss_a, o);
+            ss_b += __shfl_xor_sync(0xFFFFFFFFu, ss_b, o);
+        }
+        __syncthreads();   // everyone has read m.mu before m.red is reused
+        if (lane == 0) {
+            m.red[0][warp] = ss_a;
+            m.red[1][warp] = ss_b;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int t = 0; t < 2; ++t) {
+            double ss = 0.0;
+            for (int w = 0; w < kNumWarps; ++w) ss += m.red[t][w];
+            const double sigma = sqrt(ss / Nk);
+            double tau;
+            if (isinf(p.beta)) tau = p.beta < 0.0f ? -INFINITY : INFINITY;
+            else tau = m.mu[t] + static_cast<double>(p.beta) * sigma;
+            m.sigma[t] = sigma;
+            m.tau[t] = tau;
+        }
+        if (p.dbg_stats) {
+            for (int t = 0; t < (has_b ? 2 : 1); ++t) {
+                float *st = p.dbg_stats + (unit_a + t) * 3;
+                st[0] = static_cast<float>(m.mu[t]);
+                st[1] = static_cast<float>(m.sigma[t]);
+                st[2] = static_cast<float>(m.tau[t]);
+            }
+        }
+    }
+    __syncthreads();
+    // ---------------- routing 4: keep masks (ballot per 32 blocks), counts, debug rows
+    {
+        const double tau_a = m.tau[0], tau_b = m.tau[1];
+        const int nwords = (Nk + 31) >> 5;
+        int cnt_a = 0, cnt_b = 0;
+        for (int wd = warp; wd < nwords; wd += kNumWarps) {
+            const int j = wd * 32 + lane;
+            const bool inb = j < Nk;
+            const float sa = inb ? row_a[j] : 0.0f;
+            const float sb = inb ? row_b[j] : 0.0f;
+            const bool ka = inb && static_cast<double>(sa) >= tau_a;
+            const bool kb = inb && has_b && static_cast<double>(sb) >= tau_b;
+            const uint32_t wa = __ballot_sync(0xFFFFFFFFu, ka);
+            const uint32_t wb = __ballot_sync(0xFFFFFFFFu, kb);
+            if (lane == 0) {
+                m.mask_a[wd] = wa;
+                m.mask_b[wd] = wb;
+                m.mask_u[wd] = wa | wb;
+                cnt_a += __popc(wa);
+                cnt_b += __popc(wb);
+            }
+            if (inb) {
+                if (p.dbg_proxy) {
+                    p.dbg_proxy[unit_a * Nk + j] = sa;
+                    if (has_b) p.dbg_proxy[(unit_a + 1) * Nk + j] = sb;
+                }
+                if (p.dbg_mask) {
+                    p.dbg_mask[unit_a * Nk + j] = ka;
+                    if (has_b) p.dbg_mask[(unit_a + 1) * Nk + j] = kb;
+                }
+            }
+        }
+        if (lane == 0) {
+            atomicAdd(&m.count_a, cnt_a);
+            atomicAdd(&m.count_b, cnt_b);
+        }
+    }
+    __syncthreads();
+    // correction chunks that still hold a block skipped by tile A (or by an existing tile B)
+    {
+        const int nwords = (Nk + 31) >> 5;
+        for (int c = tid; c < p.nchunks; c += kThreads) {
+            uint32_t need = 0;
+            for (int h = 0; h < 2; ++h) {
+                const int wd = 2 * c + h;
+                if (wd >= nwords) continue;
+                const int rem = Nk - wd * 32;
+                const uint32_t valid = rem >= 32 ? 0xFFFFFFFFu : ((1u << rem) - 1u);
+                need |= valid & ~(m.mask_a[wd] & (has_b ? m.mask_b[wd] : 0xFFFFFFFFu));
+            }
+            if (need) atomicOr(&m.need[c >> 5], 1u << (c & 31));
+        }
+        if (tid == 0 && p.density) {
+            p.density[unit_a] = m.count_a;
+            if (has_b) p.density[unit_a + 1] = m.count_b;
+        }
+    }
+    fence_proxy_async_smem();   // generic writes to the ring happen-before the TMA overwrites it
+    __syncthreads();
+
+    // ---------------- pipeline
+    const bool aborted = volatile_load(&m.abort_flag) != 0;
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            if (!aborted) producer_role(&tm_k, &tm_v, &tm_kb, &tm_vb, smem, m, p, bh);
+            wait_bar(&m.q_full, 0, m, p, kSiteProdDrain, false);   // the Q copy has landed
+        }
+        __syncwarp();
+    } else if (warp == kWarpMma) {
+        if (lane == 0 && !aborted) mma_role(tmem, smem, m, p);
+        __syncwarp();
+    } else if (!aborted) {
+        softmax_role(tmem, m, p, bh, row0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
+{
+    static std::once_flag attr_once[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once[dev], [&] {
+        attr_err = cudaFuncSetAttribute(sol_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kSmemBytes));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+
+    Params p{};
+    p.BH = L.BH;
+    p.N = L.N;
+    p.Nk = L.Nk;
+    p.Nq = L.Nq;
+    p.npairs = (L.Nq + 1) / 2;
+    p.nchunks = (L.Nk + 63) / 64;
+    p.beta = L.beta;
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
+    const int n_last = L.N - (L.Nk - 1) * kTile;
+    p.last_bias_log2 = static_cast<float>(std::log2(static_cast<double>(n_last)));
+    p.kbar32 = L.kbar32;
+    p.out = static_cast<__nv_bfloat16 *>(L.out);
+    p.density = L.density;
+    p.status = L.status;
+    p.dbg_proxy = L.dbg_proxy;
+    p.dbg_mask = L.dbg_mask;
+    p.dbg_stats = L.dbg_stats;
+    p.fault_flags = L.fault_flags;
+    p.timeout_ns = L.timeout_ns;
+    const long long grid = static_cast<long long>(p.npairs) * L.BH;
+    if (grid <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    sol_fwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
+        *L.tm_q, *L.tm_k, *L.tm_v, *L.tm_kb, *L.tm_vb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace sol

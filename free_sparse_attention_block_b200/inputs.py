@@ -87,7 +87,11 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 
 def _field(rng: np.random.Generator, grid, d: int, f_max: float) -> np.ndarray:
-    """Sum of 4 random sinusoids per channel over the (T, H, W) grid -> float32 [N, d]."""
+    """Sum of 4 random sinusoids per channel over the (T, H, W) grid -> float32 [N, d].
+
+    The phase is separable, angle = a(t) + b(y) + c(x) + phi, so each term is evaluated as
+    Im(e^{i a} e^{i b} e^{i (c + phi)}) with the small per-axis exponentials broadcast over the grid.
+    """
     T, Hg, Wg = grid
     f = rng.uniform(0.0, f_max, size=(d, 4, 3))
     phi = rng.uniform(0.0, 2.0 * math.pi, size=(d, 4))
@@ -96,12 +100,12 @@ def _field(rng: np.random.Generator, grid, d: int, f_max: float) -> np.ndarray:
     x = np.arange(Wg, dtype=np.float64) / Wg
     out = np.zeros((T, Hg, Wg, d), dtype=np.float64)
     for s in range(4):
-        # separable phases: angle = a(t) + b(y) + c(x) + phi, evaluated as sin(a+b+c+phi)
-        a = 2.0 * math.pi * f[:, s, 0][None, :] * t[:, None]           # [T, d]
-        b = 2.0 * math.pi * f[:, s, 1][None, :] * y[:, None]           # [H, d]
-        c = 2.0 * math.pi * f[:, s, 2][None, :] * x[:, None] + phi[:, s][None, :]  # [W, d]
-        ab = a[:, None, :] + b[None, :, :]                             # [T, H, d]
-        out += np.sin(ab[:, :, None, :] + c[None, None, :, :])
+        ea = np.exp(2j * math.pi * f[:, s, 0][None, :] * t[:, None])                  # [T, d]
+        eb = np.exp(2j * math.pi * f[:, s, 1][None, :] * y[:, None])                  # [H, d]
+        ec = np.exp(1j * (2.0 * math.pi * f[:, s, 2][None, :] * x[:, None] + phi[:, s][None, :]))  # [W, d]
+        eab = ea[:, None, :] * eb[None, :, :]                                          # [T, H, d]
+        out += eab.real[:, :, None, :] * ec.imag[None, None, :, :]
+        out += eab.imag[:, :, None, :] * ec.real[None, None, :, :]
     return out.reshape(T * Hg * Wg, d).astype(np.float32)
 
 

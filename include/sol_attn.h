@@ -1,0 +1,114 @@
+/*
+ * sol_attn.h: C ABI of the Sol-Attn block-sparse attention forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the forward pass of "Sol-Attn: Accelerating Video Generation Inference via
+ * On-the-Fly Attention Sparsification" (Li et al., 2026).  Its routing paragraphs define the
+ * block choice: a query's pre-softmax proxy scores against key blocks are reduced to a row mean
+ * mu and standard deviation sigma, and a block is computed exactly iff its score is at least
+ * tau = mu + beta*sigma (one global beta).  The fused-operator paragraph puts routing, the exact
+ * sparse attention and an approximation of every skipped block into one online-softmax pass.
+ * Readings fixed by this library where the page is silent:
+ *   - query tiles and key blocks are T = 64 tokens; Nq = Nk = ceil(N / 64); the last tile/block
+ *     may be partial with n_j = N - 64*(Nk-1) tokens;
+ *   - routing is per query tile i: S_ij = (q_bar_i . k_bar_j) / sqrt(d) with q_bar_i, k_bar_j the
+ *     float32 means of the tile's queries / the block's keys; mu_i and population sigma_i of row i
+ *     (accumulated in double); block j is kept for tile i iff S_ij >= tau_i; beta = -inf keeps
+ *     every block, beta = +inf keeps none;
+ *   - a skipped block j contributes one softmax term to each row r of the tile, with logit
+ *     (q_r . k_bar_j)/sqrt(d) + ln(n_j) and value v_bar_j (so it adds n_j*exp(q.k_bar/sqrt d - m)
+ *     to the denominator and that weight times v_bar_j to the numerator);
+ *   - bidirectional (no causal mask), forward only.
+ *
+ * Conventions for every entry point:
+ *   - q, k, v, out: bfloat16, contiguous [B, H, N, d] (token rows of d elements), device
+ *     pointers, 16-byte aligned.  d must be 128.  1 <= N <= 524288.  B*H*ceil(Nq/2) < 2^31.
+ *   - The caller owns all memory.  The library allocates no device or host memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     stream-ordered.  sol_attn_fwd needs a prior sol_attn_pool on the same K, V and workspace,
+ *     earlier in stream order.
+ *   - Errors are returned, never thrown.  Argument errors are detected on the host before any
+ *     launch.  SOL_ERR_CUDA means a CUDA runtime/driver call or launch failed.
+ *   - Device-side failures (a pipeline wait that ran out of time) are recorded in a status word
+ *     inside the workspace; sol_attn_read_status() synchronises the stream and returns it.
+ *   - The library keeps no state between calls apart from per-device one-time set-up
+ *     (kernel attributes, the driver entry point for tensor-map encoding); it is thread-safe.
+ */
+#ifndef SOL_ATTN_H
+#define SOL_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SOL_OK = 0,
+    SOL_ERR_INVALID_ARG = 1, /* null pointer, non-positive or too large size, NaN beta */
+    SOL_ERR_UNSUPPORTED = 2, /* d != 128, N above the supported maximum */
+    SOL_ERR_ALIGNMENT = 3,   /* a tensor pointer that is not 16-byte aligned */
+    SOL_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
+    SOL_ERR_TIMEOUT = 5      /* a device pipeline wait gave up (see sol_attn_read_status) */
+} sol_status;
+
+/* Bytes of device workspace sol_attn_pool/sol_attn_fwd need for this shape: a 256-byte header
+ * (status words) followed by the pooled keys and values, float32 [B,H,Nk,d] each, and their
+ * bfloat16 copies [B,H,Nk,d] each.  Returns 0 for an invalid or unsupported shape. */
+size_t sol_attn_workspace_bytes(int B, int H, int N, int d);
+
+/* Mean-pool K and V into 64-token blocks (the k_bar_j / v_bar_j of the routing and of the
+ * correction of skipped blocks).  k_bar_j[c] = (float32 sum of k_t[c] over the block's tokens in
+ * ascending order) * (1.0f / n_j); the same for v; the bfloat16 copies are round-to-nearest-even
+ * of the float32 values.  Also clears the workspace status words.
+ * workspace: device, >= sol_attn_workspace_bytes(B,H,N,d) bytes, 256-byte aligned. */
+sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int d,
+                         void *workspace, void *stream);
+
+/* Fused Sol-Attn forward: per query tile, builds the proxy row against the pooled keys in shared
+ * memory (never in global memory), reduces it to mu/sigma, keeps the blocks at or above tau, runs
+ * exact attention over the kept blocks and one pooled term per skipped block in a single
+ * online-softmax pass, and writes out = softmax-weighted values rounded to bfloat16.
+ * beta: any non-NaN float, +-inf allowed.
+ * density_out: device int32 [B,H,Nq], number of kept blocks per query tile, or NULL.
+ * workspace: the one sol_attn_pool filled for this K, V (its status words may be written). */
+sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                        float beta, void *workspace, void *out, int32_t *density_out,
+                        void *stream);
+
+/* Test/diagnostic variant of sol_attn_fwd: the same computation plus optional debug outputs,
+ * then a stream synchronisation and a read of the device status.  Not for production use.
+ *   proxy_out  device float [B,H,Nq,Nk]: the proxy rows S_ij (or NULL)
+ *   mask_out   device uint8 [B,H,Nq,Nk]: 1 = block kept (or NULL)
+ *   stats_out  device float [B,H,Nq,3]: mu_i, sigma_i, tau_i (or NULL)
+ *   fault_flags bit 0: the MMA issuer waits on a barrier nothing signals, so the pipeline wait
+ *               runs out and the call must return SOL_ERR_TIMEOUT with the context intact.
+ *   timeout_ms: limit for each device wait; <= 0 selects the production default (2000 ms).
+ * Returns SOL_ERR_TIMEOUT if any device wait ran out, else the launch status. */
+sol_status sol_attn_fwd_debug(const void *q, const void *k, const void *v, int B, int H, int N,
+                              int d, float beta, void *workspace, void *out,
+                              int32_t *density_out, float *proxy_out, uint8_t *mask_out,
+                              float *stats_out, int fault_flags, int timeout_ms, void *stream);
+
+/* Synchronise `stream`, read the device status words in the workspace header and clear them.
+ * Returns SOL_OK, SOL_ERR_TIMEOUT (a device wait gave up) or SOL_ERR_CUDA.  If where_out is not
+ * NULL it receives an internal code naming the wait that gave up (0 if none). */
+sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream);
+
+/* One end-to-end call on host buffers: copies q, k, v from (preferably pinned) host memory into
+ * the caller's device buffers, pools, runs the forward, and copies out and density back, all
+ * queued on `stream` without synchronising.  Host buffers must stay valid until the stream
+ * reaches this point.  h_density / d_density may both be NULL. */
+sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, int B, int H,
+                             int N, int d, float beta, void *d_q, void *d_k, void *d_v,
+                             void *workspace, void *d_out, int32_t *d_density, void *h_out,
+                             int32_t *h_density, void *stream);
+
+/* Static English description of a status code. */
+const char *sol_attn_error_string(sol_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_ATTN_H */

@@ -1,0 +1,87 @@
+"""The C-ABI library loads, exports every entry point include/sol_attn.h declares, and rejects
+bad arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes as C
+import math
+import os
+import re
+
+import pytest
+
+import free_sparse_attention_block_b200 as sol
+from free_sparse_attention_block_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return sol.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "sol_attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sol_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sol_attn_workspace_bytes", "sol_attn_pool", "sol_attn_fwd",
+                     "sol_attn_fwd_debug", "sol_attn_error_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_workspace_bytes(lib):
+    B, H, N = 1, 12, 16384
+    Nk = N // 64
+    n = B * H * Nk * 128
+    got = sol.sol_attn_workspace_bytes(B, H, N, 128)
+    assert got >= 256 + n * (4 + 4 + 2 + 2) and got % 256 == 0
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 128) > 0
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 64) == 0       # d != 128 unsupported
+    assert sol.sol_attn_workspace_bytes(0, 1, 100, 128) == 0
+    assert sol.sol_attn_workspace_bytes(1, 1, 524288 + 1, 128) == 0
+
+
+def test_error_strings(lib):
+    for code in range(6):
+        assert sol.sol_attn_error_string(code)
+    assert "unknown" in sol.sol_attn_error_string(99)
+
+
+A = 0x10000          # a 256-byte aligned fake device address (never dereferenced)
+MIS = 0x10008        # 8-byte aligned only
+
+
+def fwd(lib, q=A, k=A, v=A, B=1, H=1, N=128, d=128, beta=0.5, ws=A, out=A, dens=None):
+    return lib.sol_attn_fwd(q, k, v, B, H, N, d, C.c_float(beta), ws, out, dens, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
+    (dict(N=0), 1), (dict(B=-1), 1), (dict(d=64), 2), (dict(N=524288 + 64), 2),
+    (dict(beta=math.nan), 1), (dict(k=MIS), 3), (dict(ws=A + 16), 3), (dict(dens=A + 2), 3),
+])
+def test_fwd_rejects_bad_arguments_on_host(lib, kw, expect):
+    assert fwd(lib, **kw) == expect
+
+
+def test_pool_rejects_bad_arguments_on_host(lib):
+    assert lib.sol_attn_pool(None, A, 1, 1, 128, 128, A, None) == 1
+    assert lib.sol_attn_pool(A, A, 1, 1, 128, 96, A, None) == 2
+    assert lib.sol_attn_pool(A, MIS, 1, 1, 128, 128, A, None) == 3
+    assert lib.sol_attn_pool(A, A, 1, 1, 128, 128, A + 128, None) == 3
+
+
+def test_host_entry_rejects_bad_arguments_on_host(lib):
+    f = lib.sol_attn_fwd_host
+    assert f(None, A, A, 1, 1, 128, 128, C.c_float(0.5), A, A, A, A, A, None, A, None, None) == 1
+    assert f(A, A, A, 1, 1, 128, 128, C.c_float(0.5), A, A, A, A, A, A, A, None, None) == 1
+    assert f(A, A, A, 1, 1, 128, 128, C.c_float(math.nan), A, A, A, A, A, None, A, None, None) == 1
+    assert f(A, A, A, 1, 1, 128, 128, C.c_float(0.5), MIS, A, A, A, A, None, A, None, None) == 3
