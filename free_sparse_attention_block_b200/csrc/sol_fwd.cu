@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <cstddef>
 #include <mutex>
 
 #include "internal.h"
@@ -85,18 +86,21 @@ struct Misc {
     double red[2][kNumWarps];
     double mu[2], sigma[2], tau[2];
     uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2], o_done, drain, never;
+    uint64_t s_full[2], p_full[2], o_done, o_final, drain, never;
     uint32_t mask_a[kMaskWords];
     uint32_t mask_b[kMaskWords];
     uint32_t mask_u[kMaskWords];
     uint32_t need[kChunkWords];
-    float qbar[2][kHeadDim];
+    alignas(16) float qbar[2][kHeadDim];   // read as float4
     uint32_t tmem_base;
     int abort_flag;
     int count_a, count_b;
 };
 
 constexpr uint32_t kSmemBytes = kOffMisc + sizeof(Misc) + 1024;   // + alignment slack
+static_assert(offsetof(Misc, qbar) % 16 == 0, "q_bar is read with 16-byte vector loads");
+static_assert(offsetof(Misc, q_full) % 8 == 0, "mbarriers need 8-byte alignment");
+static_assert(kOffMisc % 1024 == 0, "shared-memory tiles need 1024-byte alignment");
 
 struct Params {
     int BH, N, Nk, Nq, npairs, nchunks;
@@ -268,7 +272,7 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
             if (it > 0 && !issue_pv(it - 1, tmem, smem, m, p)) { ok = false; break; }
             ++it;
         }
-        if (ok && it > 0) issue_pv(it - 1, tmem, smem, m, p);
+        if (ok && it > 0 && issue_pv(it - 1, tmem, smem, m, p)) mma_commit(&m.o_final);
     }
     // Every MMA issued so far must finish before TMEM is freed.
     mma_commit(&m.drain);
@@ -349,6 +353,9 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
             for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
         if (__any_sync(0xFFFFFFFFu, rescale) && it > 0) {
+            // PV(it-1) must be done before O is touched.  Here exactly it-1 or it PVs have
+            // completed: s_full for item it was committed after PV(it-2) was issued, and PV(it)
+            // waits for this thread's p_full arrival; so the parity of phase it-1 is unambiguous.
             ok = wait_bar(&m.o_done, (it - 1) & 1, m, p, kSiteSoftO);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
@@ -372,7 +379,9 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
         ++it;
     }
     if (!ok || it == 0) return;
-    ok = wait_bar(&m.o_done, (it - 1) & 1, m, p, kSiteEpilogue);
+    // o_final is single-use: o_done may still have two phases outstanding here (QK of the last
+    // item is issued before PV of the one before it), so its parity cannot identify the last PV.
+    ok = wait_bar(&m.o_final, 0, m, p, kSiteEpilogue);
     ok = __all_sync(0xFFFFFFFFu, ok);
     if (!ok) return;
     tc_fence_after();
@@ -432,6 +441,7 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&m.p_full[b], 128);
         }
         mbar_init(&m.o_done, 1);
+        mbar_init(&m.o_final, 1);
         mbar_init(&m.drain, 1);
         mbar_init(&m.never, 1);
         m.abort_flag = 0;
