@@ -193,6 +193,21 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// 2^x on the FMA/ALU pipes instead of the MUFU unit.  Cody-Waite reduction with one constant:
+// n = round(x) via the 1.5*2^23 shift, f = x - n in [-1/2, 1/2]; 2^f from the degree-3 polynomial
+// whose relative error is minimax on that interval (coefficients derived by fit_exp2_poly.py,
+// max relative error 7.5e-5, ample for a bf16 probability); n is added to the exponent bits.
+// x is clamped at -125 so the result stays a normal float (2^-125 is zero for a softmax weight).
+__device__ __forceinline__ float exp2_poly(float x)
+{
+    x = fmaxf(x, -125.0f);
+    const float shift = 12582912.0f;                 // 1.5 * 2^23
+    const float t = __fadd_rn(x, shift);             // low mantissa bits hold round(x)
+    const float f = __fsub_rn(x, __fsub_rn(t, shift));
+    const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     uint32_t r;

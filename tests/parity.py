@@ -4,7 +4,8 @@ with the CPU oracle on the same seeded inputs.
 Acceptance (per query tile compared):
   - block masks identical, except blocks whose oracle proxy lies within BAND of the oracle's tau
     (near ties: counted, and the oracle output is then recomputed with the GPU's decision);
-  - mu, sigma, tau within 1e-5 absolute; proxy rows within 1e-5 absolute + 1e-6 relative;
+  - mu, sigma within 1e-5 absolute; tau within 1e-5 absolute + 1e-5 relative (large |beta|);
+    proxy rows within 1e-5 absolute + 1e-6 relative;
   - kept-block counts equal to the GPU's own mask, and to the oracle's up to near ties;
   - outputs (bf16) against the float64 oracle: max-abs <= 2e-2, mean-abs <= 5e-3.
 """
@@ -111,7 +112,8 @@ def check_parity(q, k, v, beta: float, g: dict, units: np.ndarray, report: dict 
         np.testing.assert_allclose(gs[:, 0], r["mu"], rtol=0, atol=STAT_ATOL)
         np.testing.assert_allclose(gs[:, 1], r["sigma"], rtol=0, atol=STAT_ATOL)
         fin = np.isfinite(tau)
-        np.testing.assert_allclose(gs[fin, 2], tau[fin], rtol=0, atol=STAT_ATOL)
+        # tau = mu + beta*sigma: sigma agrees to ~1e-6 relative, so large |beta| needs a relative bound
+        np.testing.assert_allclose(gs[fin, 2], tau[fin], rtol=1e-5, atol=STAT_ATOL)
         assert np.array_equal(gs[~fin, 2], tau[~fin].astype(np.float32))
         gd = g["density"].reshape(-1)[units]
         assert np.array_equal(gd, gm.sum(1).astype(np.int32))

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 from free_sparse_attention_block_b200 import inputs
-from parity import check_parity, default_units, gpu_run
+from parity import MAX_ABS, MEAN_ABS, check_parity, default_units, gpu_run
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +54,9 @@ def test_hand_worked_example(golden):
         want = np.zeros(128)
         want[0] = golden[f"out_beta_{key}_ch0"]
         want[1] = golden[f"out_beta_{key}_ch1"]
-        np.testing.assert_allclose(out, np.broadcast_to(want, out.shape), atol=4e-3)
+        err = np.abs(out - want[None, :])
+        # the suite's output bar (bf16 output and bf16 probabilities against the exact value)
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     for beta, m in [(1.0, [1, 0]), (-1.0, [1, 1])]:      # exact ties: ">=" keeps the block
         g = gpu_run(q[None], k[None], v[None], beta)
         assert g["mask"].reshape(2, 2).tolist() == [m, m]
