@@ -20,14 +20,15 @@ __all__ = [
     "SolError", "load_library", "LIB_PATH", "HEAD_DIM", "TILE", "STATUS",
     "sol_attn_workspace_bytes", "sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug",
     "sol_attn_read_status", "sol_attn_fwd_host", "sol_attn_error_string", "forward",
-    "workspace_views",
+    "workspace_views", "sol_attn_fwd_noalloc", "NOALLOC_MAX_BYTES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
 HEAD_DIM = 128
 TILE = 64
 STATUS = {0: "SOL_OK", 1: "SOL_ERR_INVALID_ARG", 2: "SOL_ERR_UNSUPPORTED", 3: "SOL_ERR_ALIGNMENT",
-          4: "SOL_ERR_CUDA", 5: "SOL_ERR_TIMEOUT"}
+          4: "SOL_ERR_CUDA", 5: "SOL_ERR_TIMEOUT", 6: "SOL_ERR_SCRATCH_LIMIT"}
+NOALLOC_MAX_BYTES = 16 * 1024 * 1024
 
 _lock = threading.Lock()
 _lib = None
@@ -58,10 +59,11 @@ def load_library(path: str | None = None):
         lib.sol_attn_fwd_debug.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp, i, i, vp]
         lib.sol_attn_read_status.argtypes = [vp, C.POINTER(C.c_int), vp]
         lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.sol_attn_fwd_noalloc.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         lib.sol_attn_error_string.argtypes = [i]
         lib.sol_attn_error_string.restype = C.c_char_p
         for name in ("sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug", "sol_attn_read_status",
-                     "sol_attn_fwd_host"):
+                     "sol_attn_fwd_host", "sol_attn_fwd_noalloc"):
             getattr(lib, name).restype = C.c_int
         if path is None:
             _lib = lib
@@ -148,6 +150,19 @@ def sol_attn_fwd_host(h_q, h_k, h_v, beta: float, d_q, d_k, d_v, workspace, d_ou
         _ptr(workspace), _ptr(d_out), _ptr(d_density), _ptr(h_out), _ptr(h_density), _stream(stream))
     if check:
         _check(st, "sol_attn_fwd_host")
+    return st
+
+
+def sol_attn_fwd_noalloc(q, k, v, beta: float, out, density_out=None, stream=None,
+                         check: bool = True) -> int:
+    """Pool + forward without a caller workspace: the library's built-in scratch (at most
+    NOALLOC_MAX_BYTES) holds the pooled keys/values.  For callers that cannot allocate device
+    memory.  Calls that overlap on the GPU share that scratch and race; serialise them."""
+    B, H, N, d = _shape(q)
+    st = load_library().sol_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(beta),
+                                             _ptr(out), _ptr(density_out), _stream(stream))
+    if check:
+        _check(st, "sol_attn_fwd_noalloc")
     return st
 
 

@@ -246,6 +246,7 @@ const char *sol_attn_error_string(sol_status status)
     case SOL_ERR_ALIGNMENT: return "pointer not aligned (tensors 16 B, workspace 256 B)";
     case SOL_ERR_CUDA: return "CUDA call or kernel launch failed";
     case SOL_ERR_TIMEOUT: return "a device pipeline wait timed out";
+    case SOL_ERR_SCRATCH_LIMIT: return "shape needs more than the no-alloc scratch (SOL_ATTN_NOALLOC_MAX_BYTES)";
     }
     return "unknown status";
 }

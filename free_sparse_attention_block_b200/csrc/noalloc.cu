@@ -1,0 +1,55 @@
+// sol_attn_fwd_noalloc: the pool + fused forward for callers that must not allocate device memory
+// (for example code that runs inside a fixed device-memory budget, a host framework whose
+// allocator may not be re-entered from this call, or a plugin that owns no allocator of its own).
+// Its scratch, the pooled keys/values and the status words that sol_attn_pool/sol_attn_fwd keep
+// in a caller-provided workspace, lives in one file-scope device array instead.
+//
+// The array is a host-side stand-in for a device symbol: host code must never pass its name to a
+// kernel.  Its device address is obtained once per device with cudaGetSymbolAddress, with that
+// device current, and cached.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "sol_attn.h"
+
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[SOL_ATTN_NOALLOC_MAX_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+void *g_addr[kMaxDevices];
+cudaError_t g_err[kMaxDevices];
+
+sol_status shape_error(int B, int H, int N, int d)
+{
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SOL_ERR_INVALID_ARG;
+    if (d != sol::kHeadDim || N > sol::kMaxBlocks * sol::kTile) return SOL_ERR_UNSUPPORTED;
+    return SOL_ERR_INVALID_ARG;
+}
+
+}  // namespace
+
+extern "C" sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const void *v, int B,
+                                           int H, int N, int d, float beta, void *out,
+                                           int32_t *density_out, void *stream)
+{
+    const size_t need = sol_attn_workspace_bytes(B, H, N, d);
+    if (need == 0) return shape_error(B, H, N, d);
+    if (need > SOL_ATTN_NOALLOC_MAX_BYTES) return SOL_ERR_SCRATCH_LIMIT;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SOL_ERR_CUDA;
+    std::call_once(g_once[dev], [dev] {
+        g_err[dev] = cudaGetSymbolAddress(&g_addr[dev], g_noalloc_scratch);
+    });
+    if (g_err[dev] != cudaSuccess || g_addr[dev] == nullptr) return SOL_ERR_CUDA;
+
+    // sol_attn_pool clears the status words and overwrites every pooled row the forward reads,
+    // so nothing left in the array by an earlier call is used.
+    sol_status st = sol_attn_pool(k, v, B, H, N, d, g_addr[dev], stream);
+    if (st != SOL_OK) return st;
+    return sol_attn_fwd(q, k, v, B, H, N, d, beta, g_addr[dev], out, density_out, stream);
+}

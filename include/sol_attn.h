@@ -49,7 +49,8 @@ typedef enum {
     SOL_ERR_UNSUPPORTED = 2, /* d != 128, N above the supported maximum */
     SOL_ERR_ALIGNMENT = 3,   /* a tensor pointer that is not 16-byte aligned */
     SOL_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
-    SOL_ERR_TIMEOUT = 5      /* a device pipeline wait gave up (see sol_attn_read_status) */
+    SOL_ERR_TIMEOUT = 5,     /* a device pipeline wait gave up (see sol_attn_read_status) */
+    SOL_ERR_SCRATCH_LIMIT = 6 /* sol_attn_fwd_noalloc: the shape needs more scratch than it has */
 } sol_status;
 
 /* Bytes of device workspace sol_attn_pool/sol_attn_fwd need for this shape: a 256-byte header
@@ -103,6 +104,32 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
                              int N, int d, float beta, void *d_q, void *d_k, void *d_v,
                              void *workspace, void *d_out, int32_t *d_density, void *h_out,
                              int32_t *h_density, void *stream);
+
+/* Bytes of scratch built into the library for sol_attn_fwd_noalloc (16 MiB, one array per GPU
+ * that loads the library, held until the process exits). */
+#define SOL_ATTN_NOALLOC_MAX_BYTES (16u * 1024u * 1024u)
+
+/* sol_attn_pool + sol_attn_fwd for callers that cannot allocate device memory: code that runs
+ * inside a fixed memory budget, a host framework whose allocator must not be called back from
+ * here, or a plugin without an allocator of its own.  The paper has no counterpart; this is a
+ * packaging of the same two kernels.  Inputs and outputs are the caller's (as for sol_attn_fwd);
+ * the pooled keys/values and status words go to a scratch array inside the library instead of a
+ * caller workspace.  This entry point calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Limit: sol_attn_workspace_bytes(B, H, N, d) <= SOL_ATTN_NOALLOC_MAX_BYTES, i.e.
+ *     B*H*ceil(N/64) <= 10922 pooled rows (a 12-head, 16384-token call fits); larger shapes
+ *     return SOL_ERR_SCRATCH_LIMIT without launching anything.
+ *   - The first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array and leaves its contents behind; each call
+ *     clears the status words and rewrites all pooled rows it reads before use.  Calls whose
+ *     execution overlaps on the GPU (different streams, or graphs launched concurrently) race on
+ *     the array: serialise them.
+ *   - Device-side wait timeouts are recorded in the scratch status words, which the caller cannot
+ *     address; use sol_attn_fwd with an own workspace to read them.
+ * Other arguments, errors and asynchrony as for sol_attn_fwd. */
+sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const void *v, int B, int H, int N,
+                                int d, float beta, void *out, int32_t *density_out, void *stream);
 
 /* Static English description of a status code. */
 const char *sol_attn_error_string(sol_status status);
