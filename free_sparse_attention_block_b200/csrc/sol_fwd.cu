@@ -46,6 +46,7 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kNumWarps = 6;
+constexpr int kSoftmaxThreads = 128;   // warps 0-3: one thread per row (TMEM lane)
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
 constexpr int kBM = 128;
@@ -61,6 +62,15 @@ constexpr uint32_t kTmemO = 128;                       // O accumulator: columns
 __device__ __forceinline__ uint32_t tmem_s_col(int b) { return b ? 64u : 0u; }
 
 constexpr float kRescaleLog2 = 8.0f;                   // rescale O only if the max grows > 2^8
+
+// Of the 32 column pairs of a row, this many take exp2 on the FMA pipe (exp2_poly2) and the rest
+// on the MUFU unit.  Measured on the mid workload (beta 0.5): 0 pairs 0.592 ms, 6: 0.601,
+// 12: 0.619, 20: 0.643 -- the MUFU unit is not the limit at this pipeline depth, so the default
+// keeps every exp2 on MUFU; the polynomial stays available for a deeper pipeline.
+#ifndef SOL_EXP2_POLY_PAIRS
+#define SOL_EXP2_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = SOL_EXP2_POLY_PAIRS;
 
 constexpr int kMaskWords = kMaxBlocks / 32;
 constexpr int kChunkWords = (kMaxBlocks / 64 + 31) / 32;
@@ -85,8 +95,8 @@ enum WaitSite : int {
 struct Misc {
     double red[2][kNumWarps];
     double mu[2], sigma[2], tau[2];
-    uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2], o_done, o_final, drain, never;
+    uint64_t q_full, k_full[kStages], v_full[kStages], v_empty[kStages];
+    uint64_t s_full[2], p_full[2], o_final, drain, never;
     uint32_t mask_a[kMaskWords];
     uint32_t mask_b[kMaskWords];
     uint32_t mask_u[kMaskWords];
@@ -185,34 +195,45 @@ __device__ __forceinline__ float bf16_at(const uint8_t *p)
 
 // ----------------------------------------------------------------------------- roles
 
+__device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int row, int bh)
+{
+    mbar_arrive_expect_tx(bar, kKVTileBytes);
+    tma_load_3d(dst, map, bar, 0, row, bh);
+    tma_load_3d(dst + kKVHalfBytes, map, bar, 64, row, bh);
+}
+
+// One thread feeds both rings.  The tensor core retires work in the order
+// QK(it-2), PV(it-3), QK(it-1), PV(it-2), ... (the MMA issuer emits QK(j) then PV(j-1)), so the
+// producer loads K(it) once QK(it-2) has freed its stage and then V(it-1) once PV(it-3) has freed
+// its stage: its blocking waits follow the completion order, and a K load never queues behind a V
+// stage that frees later.  K stage s is free when the QK of item it-2 has completed, which is the
+// phase of s_full[s] for that item (the S buffer and the K stage share the index); that phase
+// cannot be overtaken because QK(it) needs the tile loaded here.
 __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                               const CUtensorMap *tm_kb, const CUtensorMap *tm_vb, uint8_t *smem,
                               Misc &m, const Params &p, int bh)
 {
     int issued_k[kStages], issued_v[kStages];
     for (int s = 0; s < kStages; ++s) issued_k[s] = issued_v[s] = -1;
-    Walker w;
-    int it = 0;
-    while (w.next(m, p)) {
-        const int s = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        const bool corr = w.phase == 0;
-        const CUtensorMap *mk = corr ? tm_kb : tm_k;
-        const CUtensorMap *mv = corr ? tm_vb : tm_v;
-        const int row = w.idx * kTile;
-        uint8_t *kdst = smem + kOffK + s * kKVTileBytes;
-        uint8_t *vdst = smem + kOffV + s * kKVTileBytes;
-        if (!wait_bar(&m.k_empty[s], ph ^ 1u, m, p, kSiteProdK)) break;
-        mbar_arrive_expect_tx(&m.k_full[s], kKVTileBytes);
-        tma_load_3d(kdst, mk, &m.k_full[s], 0, row, bh);
-        tma_load_3d(kdst + kKVHalfBytes, mk, &m.k_full[s], 64, row, bh);
-        issued_k[s] = it;
-        if (!wait_bar(&m.v_empty[s], ph ^ 1u, m, p, kSiteProdV)) break;
-        mbar_arrive_expect_tx(&m.v_full[s], kKVTileBytes);
-        tma_load_3d(vdst, mv, &m.v_full[s], 0, row, bh);
-        tma_load_3d(vdst + kKVHalfBytes, mv, &m.v_full[s], 64, row, bh);
-        issued_v[s] = it;
-        ++it;
+    Walker wk, wv;
+    bool more_k = wk.next(m, p), more_v = wv.next(m, p);
+    bool ok = true;
+    for (int it = 0; ok && (more_k || more_v); ++it) {
+        if (more_k) {
+            const int s = it & 1;
+            if (it >= 2 && !wait_bar(&m.s_full[s], ((it - 2) >> 1) & 1, m, p, kSiteProdK)) { ok = false; break; }
+            load_tile(smem + kOffK + s * kKVTileBytes, wk.phase == 0 ? tm_kb : tm_k, &m.k_full[s], wk.idx * kTile, bh);
+            issued_k[s] = it;
+            more_k = wk.next(m, p);
+        }
+        const int iv = it - 1;
+        if (iv >= 0 && more_v) {
+            const int s = iv & 1;
+            if (iv >= 2 && !wait_bar(&m.v_empty[s], ((iv - 2) >> 1) & 1, m, p, kSiteProdV)) { ok = false; break; }
+            load_tile(smem + kOffV + s * kKVTileBytes, wv.phase == 0 ? tm_vb : tm_v, &m.v_full[s], wv.idx * kTile, bh);
+            issued_v[s] = iv;
+            more_v = wv.next(m, p);
+        }
     }
     // No TMA write may still be in flight when the CTA exits.
     for (int s = 0; s < kStages; ++s) {
@@ -221,24 +242,24 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
     }
 }
 
-__device__ __forceinline__ bool issue_pv(int t, uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
+__device__ __forceinline__ bool issue_pv(int t, uint32_t tmem, uint64_t dv0, Misc &m, const Params &p)
 {
     const int b = t & 1, s = t & 1;
     const uint32_t ph = (t >> 1) & 1;
     if (!wait_bar(&m.p_full[b], ph, m, p, kSiteMmaP)) return false;
     if (!wait_bar(&m.v_full[s], ph, m, p, kSiteMmaV)) return false;
     tc_fence_after();
-    const uint32_t v_base = smem_u32(smem + kOffV + s * kKVTileBytes);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        // B = V tile, MN-major: 64 channels contiguous per key row (128 B, swizzled), next 8 keys
-        // at +1024 B (SBO), channels 64..127 at +8192 B (LBO); 16 keys per MMA -> +2048 B.
-        const uint64_t bdesc = desc_sw128(v_base + kk * 2048, kKVHalfBytes, 1024);
-        mma_ts(tmem + kTmemO, tmem + tmem_s_col(b) + kk * 8, bdesc, kIdescPV,
-               (t > 0 || kk > 0) ? 1u : 0u);
-    }
+    // B = V tile of stage s, MN-major: 64 channels contiguous per key row (128 B, swizzled), next
+    // 8 keys at +1024 B (SBO), channels 64..127 at +8192 B (LBO); 16 keys per MMA -> +2048 B,
+    // i.e. +128 in the descriptor's 16-byte address units.
+    const uint64_t dv = dv0 + static_cast<uint64_t>(s) * (kKVTileBytes >> 4);
+    const uint32_t a0 = tmem + tmem_s_col(b);
+    if (t > 0) mma_ts_acc(tmem + kTmemO, a0, dv, kIdescPV);
+    else mma_ts(tmem + kTmemO, a0, dv, kIdescPV, 0u);
+    mma_ts_acc(tmem + kTmemO, a0 + 8, dv + 128, kIdescPV);
+    mma_ts_acc(tmem + kTmemO, a0 + 16, dv + 256, kIdescPV);
+    mma_ts_acc(tmem + kTmemO, a0 + 24, dv + 384, kIdescPV);
     mma_commit(&m.v_empty[s]);
-    mma_commit(&m.o_done);
     return true;
 }
 
@@ -249,36 +270,43 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
     if (ok) ok = wait_bar(&m.q_full, 0, m, p, kSiteQ);
     if (ok) {
         tc_fence_after();
-        const uint32_t q_base = smem_u32(smem + kOffQ);
+        // Descriptors are built once; a k-step or stage only adds a compile-time offset to the
+        // 14-bit start-address field (16-byte units; every address stays below 256 KB).
+        // A = Q (128 x 128), B = K tile (64 x 128), both K-major 128B-swizzled with 8-row groups
+        // 1024 B apart; channels 64..127 live in the second half buffer and a 16-channel step
+        // advances the start address by 32 B inside the swizzle atom.
+        const uint64_t dq = desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
+        const uint64_t dk0 = desc_sw128(smem_u32(smem + kOffK), 16, 1024);
+        const uint64_t dv0 = desc_sw128(smem_u32(smem + kOffV), kKVHalfBytes, 1024);
+        constexpr uint64_t kQh = kQHalfBytes >> 4, kKh = kKVHalfBytes >> 4;
         Walker w;
         int it = 0;
         while (ok && w.next(m, p)) {
             const int s = it & 1, b = it & 1;
             if (!wait_bar(&m.k_full[s], (it >> 1) & 1, m, p, kSiteMmaK)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t k_base = smem_u32(smem + kOffK + s * kKVTileBytes);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                // A = Q (128 x 128), B = K tile (64 x 128), both K-major 128B-swizzled with 8-row
-                // groups 1024 B apart; channels 64..127 live in the second half buffer and a
-                // 16-channel step advances the start address by 32 B inside the swizzle atom.
-                const uint32_t half = kk >> 2, koff = (kk & 3) * 32;
-                const uint64_t adesc = desc_sw128(q_base + half * kQHalfBytes + koff, 16, 1024);
-                const uint64_t bdesc = desc_sw128(k_base + half * kKVHalfBytes + koff, 16, 1024);
-                mma_ss(tmem + tmem_s_col(b), adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&m.k_empty[s]);
+            const uint64_t dk = dk0 + static_cast<uint64_t>(s) * (kKVTileBytes >> 4);
+            const uint32_t d = tmem + tmem_s_col(b);
+            mma_ss(d, dq, dk, kIdescQK, 0u);
+            mma_ss_acc(d, dq + 2, dk + 2, kIdescQK);
+            mma_ss_acc(d, dq + 4, dk + 4, kIdescQK);
+            mma_ss_acc(d, dq + 6, dk + 6, kIdescQK);
+            mma_ss_acc(d, dq + kQh, dk + kKh, kIdescQK);
+            mma_ss_acc(d, dq + kQh + 2, dk + kKh + 2, kIdescQK);
+            mma_ss_acc(d, dq + kQh + 4, dk + kKh + 4, kIdescQK);
+            mma_ss_acc(d, dq + kQh + 6, dk + kKh + 6, kIdescQK);
             mma_commit(&m.s_full[b]);
-            if (it > 0 && !issue_pv(it - 1, tmem, smem, m, p)) { ok = false; break; }
+            if (it > 0 && !issue_pv(it - 1, tmem, dv0, m, p)) { ok = false; break; }
             ++it;
         }
-        if (ok && it > 0 && issue_pv(it - 1, tmem, smem, m, p)) mma_commit(&m.o_final);
+        if (ok && it > 0 && issue_pv(it - 1, tmem, dv0, m, p)) mma_commit(&m.o_final);
     }
     // Every MMA issued so far must finish before TMEM is freed.
     mma_commit(&m.drain);
     wait_bar(&m.drain, 0, m, p, kSiteDrain, false);
 }
 
+// Softmax warps 0-3: thread r owns row r of the 128-row tile (TMEM lane r).
 __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, int row0)
 {
     const int row = threadIdx.x;                       // 0..127 == TMEM lane
@@ -303,35 +331,44 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
         const bool participate =
             w.phase == 0 || ((mymask[w.idx >> 5] >> (w.idx & 31)) & 1u);   // warp-uniform
         if (participate) {
-            uint32_t r0[32], r1[32];
-            tmem_ld32(s_addr, r0);
-            tmem_ld32(s_addr + 32, r1);
+            uint32_t r[64];
+            tmem_ld64(s_addr, r);
             tmem_wait_ld();
-            float x[64];
+            float mx;          // row max of the log2-domain logits of this item
+            uint64_t mul2;     // exp2 argument = r * mul2 - m_ref, two columns at a time
             if (w.phase == 0) {
+                // Correction chunk: column i is pooled block j0 + i with logit
+                // S*log2(e)/sqrt(d) + log2(n_j), or -inf if this row's tile kept block j (it is
+                // computed exactly) or j is past the last block.
                 const int c = w.idx;
-                const uint64_t sel = static_cast<uint64_t>(mymask[2 * c]) |
-                                     (static_cast<uint64_t>(mymask[2 * c + 1]) << 32);
                 const int j0 = c * 64;
+                uint64_t use = ~(static_cast<uint64_t>(mymask[2 * c]) |
+                                 (static_cast<uint64_t>(mymask[2 * c + 1]) << 32));
+                const int nvalid = p.Nk - j0;
+                if (nvalid < 64) use &= (1ull << nvalid) - 1ull;
+                const int last = p.Nk - 1 - j0;
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
-                    const int j = j0 + i;
-                    const float s = __uint_as_float(i < 32 ? r0[i] : r1[i - 32]);
-                    const float bias = (j == p.Nk - 1) ? p.last_bias_log2 : 6.0f;
-                    const bool use = (j < p.Nk) && !((sel >> i) & 1ull);
-                    x[i] = use ? fmaf(s, p.scale_log2, bias) : -INFINITY;
+                    const float bias = (i == last) ? p.last_bias_log2 : 6.0f;
+                    const float x = fmaf(__uint_as_float(r[i]), p.scale_log2, bias);
+                    r[i] = ((use >> i) & 1ull) ? __float_as_uint(x) : __float_as_uint(-INFINITY);
                 }
+                mul2 = f2(1.0f, 1.0f);
             } else {
+                // Kept block: exact logits; columns past the sequence end are -inf.
                 const int t0 = w.idx * kTile;
+                if (t0 + 64 > p.N) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float s = __uint_as_float(i < 32 ? r0[i] : r1[i - 32]);
-                    x[i] = (t0 + i < p.N) ? s * p.scale_log2 : -INFINITY;
+                    for (int i = 0; i < 64; ++i)
+                        if (t0 + i >= p.N) r[i] = __float_as_uint(-INFINITY);
                 }
+                mul2 = f2(p.scale_log2, p.scale_log2);
             }
-            float mx = x[0];
+            mx = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
 #pragma unroll
-            for (int i = 1; i < 64; ++i) mx = fmaxf(mx, x[i]);
+            for (int i = 3; i < 63; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            mx = fmaxf(mx, __uint_as_float(r[63]));
+            if (w.phase != 0) mx *= p.scale_log2;
             const float m_new = fmaxf(m_used, mx);
             if (m_new > m_used + kRescaleLog2) {
                 factor = ex2_approx(m_used - m_new);
@@ -339,24 +376,37 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
                 m_used = m_new;
             }
             const float mref = m_used == -INFINITY ? 0.0f : m_used;
-            float sum = 0.0f;
+            const uint64_t add2 = f2(-mref, -mref);
+            uint64_t sum2 = f2(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float e0 = ex2_approx(x[2 * i] - mref);
-                const float e1 = ex2_approx(x[2 * i + 1] - mref);
-                sum += e0 + e1;
+                const uint64_t a2 = ffma2(f2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), mul2, add2);
+                float e0, e1;
+                if (i < kPolyPairs) {
+                    exp2_poly2(a2, e0, e1);
+                } else {
+                    float a0, a1;
+                    unf2(a2, a0, a1);
+                    e0 = ex2_approx(a0);
+                    e1 = ex2_approx(a1);
+                }
+                sum2 = fadd2(sum2, f2(e0, e1));
                 pk[i] = pack_bf16x2(e0, e1);
             }
-            l = l * factor + sum;
+            float s0, s1;
+            unf2(sum2, s0, s1);
+            l = l * factor + (s0 + s1);
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
         if (__any_sync(0xFFFFFFFFu, rescale) && it > 0) {
-            // PV(it-1) must be done before O is touched.  Here exactly it-1 or it PVs have
-            // completed: s_full for item it was committed after PV(it-2) was issued, and PV(it)
-            // waits for this thread's p_full arrival; so the parity of phase it-1 is unambiguous.
-            ok = wait_bar(&m.o_done, (it - 1) & 1, m, p, kSiteSoftO);
+            // PV(it-1) must be done before O is touched; its completion is the phase
+            // (it-1)>>1 of v_empty[(it-1)&1].  Here PV(it-2) has completed (s_full for item it
+            // was committed after PV(it-2) was issued) and PV(it) waits for this thread's p_full
+            // arrival, so that barrier is either one phase short or complete: the parity is
+            // unambiguous.
+            ok = wait_bar(&m.v_empty[(it - 1) & 1], ((it - 1) >> 1) & 1, m, p, kSiteSoftO);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -379,8 +429,9 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
         ++it;
     }
     if (!ok || it == 0) return;
-    // o_final is single-use: o_done may still have two phases outstanding here (QK of the last
-    // item is issued before PV of the one before it), so its parity cannot identify the last PV.
+    // o_final is single-use: at this point two PVs may still be outstanding (the QK of the last
+    // item is issued before the PV of the one before it), so no per-stage parity identifies the
+    // last PV.
     ok = wait_bar(&m.o_final, 0, m, p, kSiteEpilogue);
     ok = __all_sync(0xFFFFFFFFu, ok);
     if (!ok) return;
@@ -432,15 +483,13 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(&m.q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&m.k_full[s], 1);
-            mbar_init(&m.k_empty[s], 1);
             mbar_init(&m.v_full[s], 1);
             mbar_init(&m.v_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&m.s_full[b], 1);
-            mbar_init(&m.p_full[b], 128);
+            mbar_init(&m.p_full[b], kSoftmaxThreads);
         }
-        mbar_init(&m.o_done, 1);
         mbar_init(&m.o_final, 1);
         mbar_init(&m.drain, 1);
         mbar_init(&m.never, 1);
@@ -499,57 +548,70 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float *row_b = reinterpret_cast<float *>(smem + kOffRowB);
     const size_t unit_a = static_cast<size_t>(bh) * p.Nq + tile_a;
     {
+        // Each warp takes groups of 8 key blocks (group g = blocks 8g..8g+7; warp w takes groups
+        // w, w+6, ...).  Lane l holds channels 4l..4l+3: it forms 16 partial dot products (8 blocks
+        // x tiles A/B) and a reduce-scatter over the lanes (16 shuffles) leaves the full sum of
+        // value (l >> 1) & 15 in lanes l and l^1.  The next group's rows are loaded before the
+        // current group is reduced.
         const float4 qa = reinterpret_cast<const float4 *>(m.qbar[0])[lane];
         const float4 qb = reinterpret_cast<const float4 *>(m.qbar[1])[lane];
         const float4 *kb = reinterpret_cast<const float4 *>(p.kbar32 + static_cast<size_t>(bh) * Nk * kHeadDim) + lane;
+        const int ngroups = (Nk + 7) >> 3;
+        const int my_idx = (lane >> 1) & 15;
         double sum_a = 0.0, sum_b = 0.0;
-        int j = warp;
-        for (; j + 3 * kNumWarps < Nk; j += 4 * kNumWarps) {
-            float4 x[4];
+        float4 x[8];
+        int g = warp;
+        if (g < ngroups) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) x[u] = __ldg(kb + static_cast<size_t>(j + u * kNumWarps) * 32);
-            float a[4], b[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                a[u] = fmaf(qa.w, x[u].w, fmaf(qa.z, x[u].z, fmaf(qa.y, x[u].y, qa.x * x[u].x)));
-                b[u] = fmaf(qb.w, x[u].w, fmaf(qb.z, x[u].z, fmaf(qb.y, x[u].y, qb.x * x[u].x)));
+            for (int u = 0; u < 8; ++u) {
+                const int j = 8 * g + u;
+                x[u] = j < Nk ? __ldg(kb + static_cast<size_t>(j) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
+        }
+        for (; g < ngroups; g += kNumWarps) {
+            float v[16];
 #pragma unroll
-            for (int o = 16; o; o >>= 1) {
+            for (int u = 0; u < 8; ++u) {
+                v[u] = fmaf(qa.w, x[u].w, fmaf(qa.z, x[u].z, fmaf(qa.y, x[u].y, qa.x * x[u].x)));
+                v[8 + u] = fmaf(qb.w, x[u].w, fmaf(qb.z, x[u].z, fmaf(qb.y, x[u].y, qb.x * x[u].x)));
+            }
+            const int gn = g + kNumWarps;
+            if (gn < ngroups) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    a[u] += __shfl_xor_sync(0xFFFFFFFFu, a[u], o);
-                    b[u] += __shfl_xor_sync(0xFFFFFFFFu, b[u], o);
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 8 * gn + u;
+                    x[u] = j < Nk ? __ldg(kb + static_cast<size_t>(j) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            if (lane == 0) {
+            float k8[8], k4[4], k2[2];
+            const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4, h2 = lane & 2;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int jj = j + u * kNumWarps;
-                    const float sa = a[u] * p.scale, sb = b[u] * p.scale;
-                    row_a[jj] = sa;
-                    row_b[jj] = sb;
-                    sum_a += sa;
-                    sum_b += sb;
+            for (int i = 0; i < 8; ++i)
+                k8[i] = (h16 ? v[i + 8] : v[i]) + __shfl_xor_sync(0xFFFFFFFFu, h16 ? v[i] : v[i + 8], 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                k4[i] = (h8 ? k8[i + 4] : k8[i]) + __shfl_xor_sync(0xFFFFFFFFu, h8 ? k8[i] : k8[i + 4], 8);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                k2[i] = (h4 ? k4[i + 2] : k4[i]) + __shfl_xor_sync(0xFFFFFFFFu, h4 ? k4[i] : k4[i + 2], 4);
+            const float k1 = (h2 ? k2[1] : k2[0]) + __shfl_xor_sync(0xFFFFFFFFu, h2 ? k2[0] : k2[1], 2);
+            const float tot = k1 + __shfl_xor_sync(0xFFFFFFFFu, k1, 1);
+            const int j = 8 * g + (my_idx & 7);
+            if ((lane & 1) == 0 && j < Nk) {
+                const float sc = tot * p.scale;
+                if (my_idx < 8) {
+                    row_a[j] = sc;
+                    sum_a += sc;
+                } else {
+                    row_b[j] = sc;
+                    sum_b += sc;
                 }
             }
         }
-        for (; j < Nk; j += kNumWarps) {
-            const float4 x = __ldg(kb + static_cast<size_t>(j) * 32);
-            float a = fmaf(qa.w, x.w, fmaf(qa.z, x.z, fmaf(qa.y, x.y, qa.x * x.x)));
-            float b = fmaf(qb.w, x.w, fmaf(qb.z, x.z, fmaf(qb.y, x.y, qb.x * x.x)));
 #pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
-                b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
-            }
-            if (lane == 0) {
-                const float sa = a * p.scale, sb = b * p.scale;
-                row_a[j] = sa;
-                row_b[j] = sb;
-                sum_a += sa;
-                sum_b += sb;
-            }
+        for (int o = 16; o; o >>= 1) {
+            sum_a += __shfl_xor_sync(0xFFFFFFFFu, sum_a, o);
+            sum_b += __shfl_xor_sync(0xFFFFFFFFu, sum_b, o);
         }
         if (lane == 0) {
             m.red[0][warp] = sum_a;
