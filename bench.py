@@ -61,7 +61,7 @@ def kernel_hash() -> str:
 # ------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML every ~10 ms (read-only)."""
+    """Samples SM clock and clock-event reasons through NVML every ~2 ms (read-only)."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -93,7 +93,7 @@ class ClockSampler:
                 self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.ok:
@@ -112,6 +112,25 @@ class ClockSampler:
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
         return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ multi-GPU timing
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Slowest rank's value (device-timed milliseconds) when a process group is up, else x."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(dense_flops_per_replica: float, world: int, t_max_ms: float) -> float:
+    """Whole-job dense-equivalent TFLOP/s of `world` independent replicas over the slowest rank's
+    time (weak scaling: each rank runs the full workload)."""
+    return world * dense_flops_per_replica / (t_max_ms * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------------------ flops
@@ -305,14 +324,9 @@ def run_ours(args, wl):
         raise RuntimeError(f"device status {sol.STATUS.get(st)} at wait site {where}")
 
     # max over ranks of the device time
-    t_max = step_ms
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-
+    t_max = max_over_ranks(step_ms, dev)
     dense = wl.dense_flops()
-    value = world * dense / (t_max * 1e-3) / 1e12
+    value = replica_throughput(dense, world, t_max)
 
     # ---- e2e through the C ABI on pinned host buffers (copies inside the timed region)
     hq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -330,11 +344,7 @@ def run_ours(args, wl):
         sol.sol_attn_fwd_host(hq, hk, hv, args.beta, tq, tk, tv, ws, out, hout, dens, hdens)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     assert torch.isfinite(hout.float()).all()
     h2d = 3 * B * H * N * d * 2
     d2h = B * H * N * d * 2 + B * H * Nq * 4
@@ -342,7 +352,8 @@ def run_ours(args, wl):
     # ---- beta sweep (fwd only, same inputs), for the record
     sweep = []
     if args.sweep:
-        for beta in wl.betas:
+        # the workload's beta sweep, plus 0.25 and 0.0 so that densities of 0.3 and above are covered
+        for beta in sorted(set(wl.betas) | {0.0, 0.25}):
             m2 = torch.empty((B, H, Nq, Nq), dtype=torch.uint8, device=dev)
             sol.sol_attn_fwd_debug(tq, tk, tv, beta, ws, out, dens, None, m2, None)
             fc2 = flop_counts(m2.cpu().numpy().reshape(B * H, Nq, Nq), N, d)
@@ -396,7 +407,7 @@ def run_ours(args, wl):
                      "peak_source": f"bf16_tflops ({PEAK_SRC}; burst)", "kernel": "sol_fwd_kernel",
                      "algorithmic_flops_per_launch": fc["kept"] + fc["corr"]},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms": e2e_ms,
+        "e2e": {"value": replica_throughput(dense, world, e2e_ms), "unit": UNIT, "ms": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "sol_attn_fwd_host (pinned host buffers)"},
         "gpu_launches": 2 * args.steps,

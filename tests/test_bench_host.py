@@ -1,0 +1,54 @@
+"""Host-side logic of bench.py (no GPU): the flop accounting from a block mask, and the multi-GPU
+replica timing (slowest rank over a 2-rank gloo process group)."""
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_flop_counts_hand_computed():
+    # one head, N = 64*3 + 16 -> blocks of 64, 64, 64, 16; 4 query tiles (last one 16 rows)
+    N = 208
+    mask = np.zeros((1, 4, 4), np.uint8)
+    mask[0, 0, 0] = 1                       # tile 0 keeps block 0
+    mask[0, 3, 3] = 1                       # the 16-row tile keeps the 16-token block
+    mask[0, 1, :] = 1                       # tile 1 keeps everything
+    fc = bench.flop_counts(mask, N, d=128)
+    n = np.array([64, 64, 64, 16], float)
+    kept = 4 * 128 * (64 * 64 + 16 * 16 + 64 * n.sum())
+    corr = 4 * 128 * (64 * 3 + 16 * 3 + 64 * 4)   # skipped pairs: tile0 3, tile3 3, tile2 4
+    assert fc["kept"] == kept and fc["corr"] == corr
+    assert fc["density"] == mask.mean()
+    # tile pairs (0,1) and (2,3): unions of 4 and 1 kept blocks; one correction chunk each
+    # (tile 0 and tile 2 skip blocks) -> 7 MMA iterations of 128 x 64 keys
+    assert fc["executed"] == 4 * 128 * 128 * 64 * (4 + 1 + 2)
+
+
+def test_replica_throughput():
+    assert bench.replica_throughput(1e12, 1, 1.0) == 1000.0
+    assert bench.replica_throughput(1e12, 4, 2.0) == 2000.0
+
+
+def _worker(rank, world, port, times, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out[rank] = bench.max_over_ranks(times[rank], "cpu")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    times = [1.25, 3.5]
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_worker, args=(2, port, times, out), nprocs=2, start_method="spawn", join=True)
+    assert out[0] == out[1] == 3.5
+    assert bench.max_over_ranks(2.0) == 2.0        # no process group: unchanged
