@@ -20,7 +20,7 @@ __all__ = [
     "SolError", "load_library", "LIB_PATH", "HEAD_DIM", "TILE", "STATUS",
     "sol_attn_workspace_bytes", "sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug",
     "sol_attn_read_status", "sol_attn_fwd_host", "sol_attn_error_string", "forward",
-    "workspace_views", "sol_attn_fwd_noalloc", "NOALLOC_MAX_BYTES",
+    "workspace_views", "sol_attn_fwd_noalloc", "NOALLOC_MAX_BYTES", "sol_attn_fwd_betas",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
@@ -60,10 +60,11 @@ def load_library(path: str | None = None):
         lib.sol_attn_read_status.argtypes = [vp, C.POINTER(C.c_int), vp]
         lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.sol_attn_fwd_noalloc.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp]
+        lib.sol_attn_fwd_betas.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
         lib.sol_attn_error_string.argtypes = [i]
         lib.sol_attn_error_string.restype = C.c_char_p
         for name in ("sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug", "sol_attn_read_status",
-                     "sol_attn_fwd_host", "sol_attn_fwd_noalloc"):
+                     "sol_attn_fwd_host", "sol_attn_fwd_noalloc", "sol_attn_fwd_betas"):
             getattr(lib, name).restype = C.c_int
         if path is None:
             _lib = lib
@@ -122,6 +123,20 @@ def sol_attn_fwd(q, k, v, beta: float, workspace, out, density_out=None, stream=
                                      _ptr(workspace), _ptr(out), _ptr(density_out), _stream(stream))
     if check:
         _check(st, "sol_attn_fwd")
+    return st
+
+
+def sol_attn_fwd_betas(q, k, v, beta_per_head, workspace, out, density_out=None, stream=None,
+                       check: bool = True) -> int:
+    """sol_attn_fwd with one beta per head: beta_per_head is a float32 device tensor of B*H."""
+    B, H, N, d = _shape(q)
+    if beta_per_head.numel() != B * H:
+        raise ValueError("beta_per_head must hold B*H values")
+    st = load_library().sol_attn_fwd_betas(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(beta_per_head),
+                                           _ptr(workspace), _ptr(out), _ptr(density_out),
+                                           _stream(stream))
+    if check:
+        _check(st, "sol_attn_fwd_betas")
     return st
 
 

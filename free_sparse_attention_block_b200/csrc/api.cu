@@ -92,8 +92,8 @@ bool encode_rows(CUtensorMap *map, const void *base, long long rows, int BH, int
 }
 
 sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
-                   float beta, void *workspace, void *out, int32_t *density, float *dbg_proxy,
-                   uint8_t *dbg_mask, float *dbg_stats, int fault_flags,
+                   float beta, const float *beta_head, void *workspace, void *out, int32_t *density,
+                   float *dbg_proxy, uint8_t *dbg_mask, float *dbg_stats, int fault_flags,
                    unsigned long long timeout_ns, cudaStream_t stream)
 {
     Shape s{};
@@ -104,6 +104,7 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     if (st != SOL_OK) return st;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
     if (density && (reinterpret_cast<uintptr_t>(density) & 3u)) return SOL_ERR_ALIGNMENT;
+    if (beta_head && (reinterpret_cast<uintptr_t>(beta_head) & 3u)) return SOL_ERR_ALIGNMENT;
 
     const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -123,6 +124,7 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     L.Nk = s.Nk;
     L.Nq = s.Nq;
     L.beta = beta;
+    L.beta_head = beta_head;
     L.kbar32 = reinterpret_cast<const float *>(ws + wl.kbar32);
     L.out = out;
     L.density = density;
@@ -173,8 +175,17 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
 sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
                         float beta, void *workspace, void *out, int32_t *density_out, void *stream)
 {
-    return run_fwd(q, k, v, B, H, N, d, beta, workspace, out, density_out, nullptr, nullptr,
-                   nullptr, 0, kDefaultTimeoutNs, static_cast<cudaStream_t>(stream));
+    return run_fwd(q, k, v, B, H, N, d, beta, nullptr, workspace, out, density_out, nullptr,
+                   nullptr, nullptr, 0, kDefaultTimeoutNs, static_cast<cudaStream_t>(stream));
+}
+
+sol_status sol_attn_fwd_betas(const void *q, const void *k, const void *v, int B, int H, int N,
+                              int d, const float *beta_per_head, void *workspace, void *out,
+                              int32_t *density_out, void *stream)
+{
+    if (!beta_per_head) return SOL_ERR_INVALID_ARG;
+    return run_fwd(q, k, v, B, H, N, d, 0.0f, beta_per_head, workspace, out, density_out, nullptr,
+                   nullptr, nullptr, 0, kDefaultTimeoutNs, static_cast<cudaStream_t>(stream));
 }
 
 sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream)
@@ -200,8 +211,8 @@ sol_status sol_attn_fwd_debug(const void *q, const void *k, const void *v, int B
     const unsigned long long tns =
         timeout_ms > 0 ? static_cast<unsigned long long>(timeout_ms) * 1000000ull : kDefaultTimeoutNs;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    sol_status st = run_fwd(q, k, v, B, H, N, d, beta, workspace, out, density_out, proxy_out,
-                            mask_out, stats_out, fault_flags, tns, cs);
+    sol_status st = run_fwd(q, k, v, B, H, N, d, beta, nullptr, workspace, out, density_out,
+                            proxy_out, mask_out, stats_out, fault_flags, tns, cs);
     if (st != SOL_OK) return st;
     return sol_attn_read_status(workspace, nullptr, stream);
 }

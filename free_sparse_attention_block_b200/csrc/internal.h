@@ -32,6 +32,7 @@ struct FwdLaunch {
     const CUtensorMap *tm_q, *tm_k, *tm_v, *tm_kb, *tm_vb;
     int BH, N, Nk, Nq;
     float beta;
+    const float *beta_head;   // device [BH] or null
     const float *kbar32;
     void *out;
     int32_t *density;

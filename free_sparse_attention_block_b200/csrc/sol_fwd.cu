@@ -115,6 +115,7 @@ static_assert(kOffMisc % 1024 == 0, "shared-memory tiles need 1024-byte alignmen
 struct Params {
     int BH, N, Nk, Nq, npairs, nchunks;
     float beta;
+    const float *beta_head;  // per-head beta [BH] (device) or null: then beta for every head
     float scale;           // (float)(1/sqrt(d)) for the proxy
     float scale_log2;      // log2(e)/sqrt(d) for the softmax
     float last_bias_log2;  // log2(n_last) for the last (possibly partial) block
@@ -654,8 +655,9 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int w = 0; w < kNumWarps; ++w) ss += m.red[t][w];
             const double sigma = sqrt(ss / Nk);
             double tau;
-            if (isinf(p.beta)) tau = p.beta < 0.0f ? -INFINITY : INFINITY;
-            else tau = m.mu[t] + static_cast<double>(p.beta) * sigma;
+            const float beta = p.beta_head ? p.beta_head[bh] : p.beta;
+            if (isinf(beta)) tau = beta < 0.0f ? -INFINITY : INFINITY;
+            else tau = m.mu[t] + static_cast<double>(beta) * sigma;   // NaN beta: NaN tau, nothing kept
             m.sigma[t] = sigma;
             m.tau[t] = tau;
         }
@@ -775,6 +777,7 @@ cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
     p.npairs = (L.Nq + 1) / 2;
     p.nchunks = (L.Nk + 63) / 64;
     p.beta = L.beta;
+    p.beta_head = L.beta_head;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
     const int n_last = L.N - (L.Nk - 1) * kTile;

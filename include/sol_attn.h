@@ -77,6 +77,15 @@ sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int 
                         float beta, void *workspace, void *out, int32_t *density_out,
                         void *stream);
 
+/* sol_attn_fwd with one beta per head: beta_per_head is a device float array [B*H] (index
+ * b*H + h), 4-byte aligned.  Entries may be +-inf; a NaN entry gives a NaN threshold, so that
+ * head keeps no block.  This is the per-head form of the threshold paragraph's single global
+ * offset, used to hold every head at the same target density (see the Python helper
+ * calibrate_betas). */
+sol_status sol_attn_fwd_betas(const void *q, const void *k, const void *v, int B, int H, int N,
+                              int d, const float *beta_per_head, void *workspace, void *out,
+                              int32_t *density_out, void *stream);
+
 /* Test/diagnostic variant of sol_attn_fwd: the same computation plus optional debug outputs,
  * then a stream synchronisation and a read of the device status.  Not for production use.
  *   proxy_out  device float [B,H,Nq,Nk]: the proxy rows S_ij (or NULL)
