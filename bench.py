@@ -17,6 +17,7 @@ all ranks over the slowest rank's time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -37,7 +38,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FLUSH_BYTES = 256 << 20
 
 # DRAM bytes (read + write) per launch of the fused kernel from one ncu capture, keyed by
-# workload and beta, valid only for the kernel source whose sha256 prefix is given.
+# (workload, head dim, beta), valid only for the kernel source whose sha256 prefix is given.
 NCU_TRAFFIC = {}
 
 
@@ -146,7 +147,9 @@ def flop_counts(mask: np.ndarray, N: int, d: int = 128):
     """Algorithmic flops of one call from the block mask [BH, Nq, Nk] (uint8):
     kept = 4 d sum_{kept (i,j)} n_i n_j; correction = 4 d sum_{skipped (i,j)} n_i;
     executed = what the 128x64 MMA tiles of the kernel actually run (union of a tile pair's kept
-    blocks, plus the correction chunks it needs)."""
+    blocks, plus the correction chunks it needs).
+    density = kept blocks / all (tile, block) pairs; density_tokens = the fraction of the N^2
+    (query, key) pairs that are computed exactly (a ragged last tile/block weighs n_i n_j)."""
     n = block_lengths(N).astype(np.float64)
     m = mask.astype(bool)
     kept = 4.0 * d * float(np.einsum("bij,i,j->", m, n, n))
@@ -161,7 +164,9 @@ def flop_counts(mask: np.ndarray, N: int, d: int = 128):
     both = np.concatenate([a & b, pad], axis=2).reshape(BH, a.shape[1], nchunks, 64)
     corr_chunks = (~both.all(axis=3)).sum()
     executed = 4.0 * d * 128 * 64 * float(union + corr_chunks)
-    return dict(kept=kept, corr=corr, executed=executed, density=float(mask.mean()))
+    density_tokens = kept / (4.0 * d * BH * float(N) ** 2)
+    return dict(kept=kept, corr=corr, executed=executed, density=float(mask.mean()),
+                density_tokens=density_tokens)
 
 
 # ------------------------------------------------------------------------------ oracle arm
@@ -368,7 +373,8 @@ def run_ours(args, wl):
                 ts.append((a, b))
             torch.cuda.synchronize()
             ms = float(np.mean([a.elapsed_time(b) for a, b in ts]))
-            sweep.append({"beta": beta, "density": round(fc2["density"], 4), "fwd_ms": round(ms, 4),
+            sweep.append({"beta": beta, "density": round(fc2["density"], 4),
+                          "density_tokens": round(fc2["density_tokens"], 4), "fwd_ms": round(ms, 4),
                           "dense_equiv_tflops": round(dense / (ms * 1e-3) / 1e12, 1),
                           "computed_tile_frac": round(fc2["kept"] / (ms * 1e-3) / 1e12 / PEAK_BF16, 4)})
 
@@ -388,7 +394,7 @@ def run_ours(args, wl):
 
     achieved = (fc["kept"] + fc["corr"]) / (mean_fwd * 1e-3) / 1e12
     kh = kernel_hash()
-    tr = NCU_TRAFFIC.get((wl.name, args.beta))
+    tr = NCU_TRAFFIC.get((wl.name, wl.d, args.beta))
     traffic = tr["bytes"] if tr and tr["kernel"] == kh else None
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -398,6 +404,7 @@ def run_ours(args, wl):
         "fwd_ms": mean_fwd, "pool_ms": mean_pool,
         "pool_gbs": (2 * B * H * N * d * 2 + B * H * Nq * d * 12) / (mean_pool * 1e-3) / 1e9,
         "density": fc["density"],
+        "density_tokens": fc["density_tokens"],
         "computed_tile_frac": fc["kept"] / (mean_fwd * 1e-3) / 1e12 / PEAK_BF16,
         "computed_tile_frac_sustained": fc["kept"] / (mean_fwd * 1e-3) / 1e12 / PEAK_BF16_SUST,
         "executed_mma_tflops": fc["executed"] / (mean_fwd * 1e-3) / 1e12,
@@ -437,9 +444,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU-baseline sample time")
     ap.add_argument("--ref-seconds", type=float, default=90.0, help="target total time of the oracle arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head-dim", type=int, choices=[64, 128], default=None,
+                    help="generate the workload with this head dimension instead of its own")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = inputs.WORKLOADS[args.workload]
+    if args.head_dim is not None and args.head_dim != wl.d:
+        wl = dataclasses.replace(wl, d=args.head_dim, name=f"{wl.name}_d{args.head_dim}")
     if args.impl == "reference":
         run_reference(args, wl)
     else:

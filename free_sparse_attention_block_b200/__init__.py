@@ -6,7 +6,7 @@ kernels of ``libsolattn.so``.  There is no CPU or PyTorch fallback; if the libra
 first call raises.
 
     import torch, free_sparse_attention_block_b200 as sol
-    out, density = sol.forward(q, k, v, beta=0.5)      # q, k, v: bf16 [B, H, N, 128] on cuda
+    out, density = sol.forward(q, k, v, beta=0.5)      # q, k, v: bf16 [B, H, N, d] on cuda, d = 64 or 128
 
 The functions named ``sol_attn_*`` mirror the C entry points one to one.
 """
@@ -17,14 +17,15 @@ import os
 import threading
 
 __all__ = [
-    "SolError", "load_library", "LIB_PATH", "HEAD_DIM", "TILE", "STATUS",
+    "SolError", "load_library", "LIB_PATH", "HEAD_DIM", "HEAD_DIMS", "TILE", "STATUS",
     "sol_attn_workspace_bytes", "sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug",
     "sol_attn_read_status", "sol_attn_fwd_host", "sol_attn_error_string", "forward",
     "workspace_views", "sol_attn_fwd_noalloc", "NOALLOC_MAX_BYTES", "sol_attn_fwd_betas",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
-HEAD_DIM = 128
+HEAD_DIM = 128              # default head dimension; HEAD_DIMS lists every compiled one
+HEAD_DIMS = (64, 128)
 TILE = 64
 STATUS = {0: "SOL_OK", 1: "SOL_ERR_INVALID_ARG", 2: "SOL_ERR_UNSUPPORTED", 3: "SOL_ERR_ALIGNMENT",
           4: "SOL_ERR_CUDA", 5: "SOL_ERR_TIMEOUT", 6: "SOL_ERR_SCRATCH_LIMIT"}
@@ -181,18 +182,18 @@ def sol_attn_fwd_noalloc(q, k, v, beta: float, out, density_out=None, stream=Non
     return st
 
 
-def workspace_views(workspace, B: int, H: int, N: int):
+def workspace_views(workspace, B: int, H: int, N: int, d: int = HEAD_DIM):
     """Views of the pooled arrays inside a workspace tensor (uint8, device): (kbar32, vbar32,
-    kbar16, vbar16) shaped [B, H, Nk, 128]; the layout mirrors the C library's."""
+    kbar16, vbar16) shaped [B, H, Nk, d]; the layout mirrors the C library's."""
     import torch
     Nk = (N + TILE - 1) // TILE
-    n = B * H * Nk * HEAD_DIM
+    n = B * H * Nk * d
     up = lambda x: (x + 255) & ~255
     o_k32 = 256
     o_v32 = up(o_k32 + 4 * n)
     o_k16 = up(o_v32 + 4 * n)
     o_v16 = up(o_k16 + 2 * n)
-    shp = (B, H, Nk, HEAD_DIM)
+    shp = (B, H, Nk, d)
     k32 = workspace[o_k32:o_k32 + 4 * n].view(torch.float32).view(shp)
     v32 = workspace[o_v32:o_v32 + 4 * n].view(torch.float32).view(shp)
     k16 = workspace[o_k16:o_k16 + 2 * n].view(torch.bfloat16).view(shp)

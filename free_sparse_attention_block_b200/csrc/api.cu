@@ -12,10 +12,10 @@
 
 namespace sol {
 
-WorkspaceLayout workspace_layout(long long BH, long long Nk)
+WorkspaceLayout workspace_layout(long long BH, long long Nk, int d)
 {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t elems = static_cast<size_t>(BH) * static_cast<size_t>(Nk) * kHeadDim;
+    const size_t elems = static_cast<size_t>(BH) * static_cast<size_t>(Nk) * static_cast<size_t>(d);
     WorkspaceLayout w{};
     w.kbar32 = kHeaderBytes;
     w.vbar32 = up(w.kbar32 + elems * 4);
@@ -30,13 +30,13 @@ namespace {
 constexpr int kMaxN = kMaxBlocks * kTile;   // 524288
 
 struct Shape {
-    int BH, N, Nk, Nq;
+    int BH, N, Nk, Nq, d;
 };
 
 sol_status check_shape(int B, int H, int N, int d, Shape *s)
 {
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SOL_ERR_INVALID_ARG;
-    if (d != kHeadDim) return SOL_ERR_UNSUPPORTED;
+    if (!head_dim_supported(d)) return SOL_ERR_UNSUPPORTED;
     if (N > kMaxN) return SOL_ERR_UNSUPPORTED;
     const long long BH = static_cast<long long>(B) * H;
     const long long Nk = (N + kTile - 1) / kTile;
@@ -45,6 +45,7 @@ sol_status check_shape(int B, int H, int N, int d, Shape *s)
     s->N = N;
     s->Nk = static_cast<int>(Nk);
     s->Nq = static_cast<int>(Nk);
+    s->d = d;
     return SOL_OK;
 }
 
@@ -73,16 +74,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// 3-D bf16 map over [BH][rows][128] with a {64 channels, box_rows} box, 128-byte swizzle and
+// 3-D bf16 map over [BH][rows][d] with a {64 channels, box_rows} box, 128-byte swizzle and
 // zero fill outside the tensor (rows past the end read as 0).
-bool encode_rows(CUtensorMap *map, const void *base, long long rows, int BH, int box_rows)
+bool encode_rows(CUtensorMap *map, const void *base, long long rows, int BH, int box_rows, int d)
 {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows),
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
-                             static_cast<cuuint64_t>(rows) * kHeadDim * 2};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                             static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(d) * 2};
     cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
@@ -106,12 +107,13 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     if (density && (reinterpret_cast<uintptr_t>(density) & 3u)) return SOL_ERR_ALIGNMENT;
     if (beta_head && (reinterpret_cast<uintptr_t>(beta_head) & 3u)) return SOL_ERR_ALIGNMENT;
 
-    const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk);
+    const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk, s.d);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     CUtensorMap tq, tk, tv, tkb, tvb;
-    if (!encode_rows(&tq, q, s.N, s.BH, 128) || !encode_rows(&tk, k, s.N, s.BH, kTile) ||
-        !encode_rows(&tv, v, s.N, s.BH, kTile) || !encode_rows(&tkb, ws + wl.kbar16, s.Nk, s.BH, kTile) ||
-        !encode_rows(&tvb, ws + wl.vbar16, s.Nk, s.BH, kTile))
+    if (!encode_rows(&tq, q, s.N, s.BH, 128, s.d) || !encode_rows(&tk, k, s.N, s.BH, kTile, s.d) ||
+        !encode_rows(&tv, v, s.N, s.BH, kTile, s.d) ||
+        !encode_rows(&tkb, ws + wl.kbar16, s.Nk, s.BH, kTile, s.d) ||
+        !encode_rows(&tvb, ws + wl.vbar16, s.Nk, s.BH, kTile, s.d))
         return SOL_ERR_CUDA;
     FwdLaunch L{};
     L.tm_q = &tq;
@@ -123,6 +125,7 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     L.N = s.N;
     L.Nk = s.Nk;
     L.Nq = s.Nq;
+    L.d = s.d;
     L.beta = beta;
     L.beta_head = beta_head;
     L.kbar32 = reinterpret_cast<const float *>(ws + wl.kbar32);
@@ -150,7 +153,7 @@ size_t sol_attn_workspace_bytes(int B, int H, int N, int d)
 {
     Shape s{};
     if (check_shape(B, H, N, d, &s) != SOL_OK) return 0;
-    return workspace_layout(s.BH, s.Nk).total;
+    return workspace_layout(s.BH, s.Nk, s.d).total;
 }
 
 sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int d,
@@ -163,10 +166,10 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
     if (st != SOL_OK) return st;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk);
+    const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk, s.d);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if (cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), cs) != cudaSuccess) return SOL_ERR_CUDA;
-    cudaError_t e = launch_pool_kv(k, v, s.BH, s.N, s.Nk, reinterpret_cast<float *>(ws + wl.kbar32),
+    cudaError_t e = launch_pool_kv(k, v, s.BH, s.N, s.Nk, s.d, reinterpret_cast<float *>(ws + wl.kbar32),
                                    reinterpret_cast<float *>(ws + wl.vbar32), ws + wl.kbar16,
                                    ws + wl.vbar16, cs);
     return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
@@ -231,7 +234,7 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
     if (st != SOL_OK) return st;
     if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    const size_t bytes = static_cast<size_t>(s.BH) * s.N * kHeadDim * 2;
+    const size_t bytes = static_cast<size_t>(s.BH) * s.N * s.d * 2;
     if (cudaMemcpyAsync(d_q, h_q, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
         cudaMemcpyAsync(d_k, h_k, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
         cudaMemcpyAsync(d_v, h_v, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
@@ -253,7 +256,7 @@ const char *sol_attn_error_string(sol_status status)
     switch (status) {
     case SOL_OK: return "success";
     case SOL_ERR_INVALID_ARG: return "invalid argument (null pointer, bad size or NaN beta)";
-    case SOL_ERR_UNSUPPORTED: return "unsupported shape (head dim must be 128, N <= 524288)";
+    case SOL_ERR_UNSUPPORTED: return "unsupported shape (head dim must be 64 or 128, N <= 524288)";
     case SOL_ERR_ALIGNMENT: return "pointer not aligned (tensors 16 B, workspace 256 B)";
     case SOL_ERR_CUDA: return "CUDA call or kernel launch failed";
     case SOL_ERR_TIMEOUT: return "a device pipeline wait timed out";

@@ -8,9 +8,10 @@
 
 namespace sol {
 
-constexpr int kHeadDim = 128;        // d
+constexpr int kMaxHeadDim = 128;     // head dimensions d = 64 and d = 128 are compiled
+inline bool head_dim_supported(int d) { return d == 64 || d == 128; }
 constexpr int kTile = 64;            // query tile / key block length T
-constexpr int kMaxBlocks = 8192;     // Nk limit: two proxy rows must fit the 64 KB K/V ring
+constexpr int kMaxBlocks = 8192;     // Nk limit: two float proxy rows (64 KB) in shared memory
 constexpr size_t kHeaderBytes = 256; // workspace header (status words)
 
 // Device status words (first bytes of the workspace header).
@@ -23,14 +24,14 @@ struct DeviceStatus {
 struct WorkspaceLayout {
     size_t kbar32, vbar32, kbar16, vbar16, total;
 };
-WorkspaceLayout workspace_layout(long long BH, long long Nk);
+WorkspaceLayout workspace_layout(long long BH, long long Nk, int d);
 
-cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, float *kbar32,
+cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, int d, float *kbar32,
                            float *vbar32, void *kbar16, void *vbar16, cudaStream_t stream);
 
 struct FwdLaunch {
     const CUtensorMap *tm_q, *tm_k, *tm_v, *tm_kb, *tm_vb;
-    int BH, N, Nk, Nq;
+    int BH, N, Nk, Nq, d;
     float beta;
     const float *beta_head;   // device [BH] or null
     const float *kbar32;

@@ -26,7 +26,7 @@ cudaError_t g_err[kMaxDevices];
 sol_status shape_error(int B, int H, int N, int d)
 {
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SOL_ERR_INVALID_ARG;
-    if (d != sol::kHeadDim || N > sol::kMaxBlocks * sol::kTile) return SOL_ERR_UNSUPPORTED;
+    if (!sol::head_dim_supported(d) || N > sol::kMaxBlocks * sol::kTile) return SOL_ERR_UNSUPPORTED;
     return SOL_ERR_INVALID_ARG;
 }
 

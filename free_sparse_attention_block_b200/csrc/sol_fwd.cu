@@ -8,8 +8,9 @@
 // sparse attention, and skipped blocks are approximated rather than dropped).
 //
 // One CTA owns one 128-row MMA tile = two adjacent 64-row routing tiles (A: rows 0-63, B: rows
-// 64-127) of one head.  Two CTAs fit on an SM (about 104 KB of shared memory and 256 TMEM
-// columns each), so one CTA's routing and softmax overlap the other's tensor-core work.
+// 64-127) of one head.  Two CTAs fit on an SM (at most about 104 KB of shared memory and 256 TMEM
+// columns each), so one CTA's routing and softmax overlap the other's tensor-core work.  The
+// kernel is compiled for head dimensions d = 128 and d = 64 (template parameter D).
 //
 //  1. Routing (all 6 warps).  TMA brings the Q tile into shared memory; q_bar of each routing
 //     tile is summed from it in float32; every warp computes proxy scores
@@ -19,9 +20,9 @@
 //     The proxy rows never reach global memory (except through the debug outputs).
 //  2. Pipeline.  Work items are first the 64-wide chunks of pooled blocks that still hold a
 //     skipped block (the correction), then every block kept by tile A or tile B (the exact part).
-//     Warp 4 (one lane) streams the item's 64x128 K and V tiles by TMA into a 2-stage ring.
-//     Warp 5 (one lane) issues S = Q K^T (M=128, N=64, K=128) into TMEM, and once the softmax has
-//     written P, O += P V (M=128, N=128, K=64) with P read straight from TMEM.
+//     Warp 4 (one lane) streams the item's 64 x d K and V tiles by TMA into a 2-stage ring.
+//     Warp 5 (one lane) issues S = Q K^T (M=128, N=64, K=d) into TMEM, and once the softmax has
+//     written P, O += P V (M=128, N=d, K=64) with P read straight from TMEM.
 //     Warps 0-3 (one thread per row) load S from TMEM, apply the per-row routing decision
 //     (a row of tile A ignores blocks only tile B kept, and vice versa; a correction column is
 //     -inf if the row's tile kept that block, else its logit gets + log2(n_j)), keep a running
@@ -52,13 +53,11 @@ constexpr int kWarpMma = 5;
 constexpr int kBM = 128;
 
 constexpr uint32_t kQHalfBytes = kBM * 64 * 2;         // 128 rows x 64 channels, bf16
-constexpr uint32_t kQBytes = 2 * kQHalfBytes;
 constexpr uint32_t kKVHalfBytes = kTile * 64 * 2;      // 64 rows x 64 channels, bf16
-constexpr uint32_t kKVTileBytes = 2 * kKVHalfBytes;
 constexpr int kStages = 2;
 
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemO = 128;                       // O accumulator: columns 128..255
+constexpr uint32_t kTmemO = 128;                       // O accumulator: columns 128..128+d-1
 __device__ __forceinline__ uint32_t tmem_s_col(int b) { return b ? 64u : 0u; }
 
 constexpr float kRescaleLog2 = 8.0f;                   // rescale O only if the max grows > 2^8
@@ -75,16 +74,29 @@ constexpr int kPolyPairs = SOL_EXP2_POLY_PAIRS;
 constexpr int kMaskWords = kMaxBlocks / 32;
 constexpr int kChunkWords = (kMaxBlocks / 64 + 31) / 32;
 
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kKVTileBytes;
-constexpr uint32_t kOffMisc = kOffV + kStages * kKVTileBytes;
-constexpr uint32_t kOffRowA = kOffK;                   // proxy rows alias the K/V ring
-constexpr uint32_t kOffRowB = kOffK + kMaxBlocks * 4;
-static_assert(kOffRowB + kMaxBlocks * 4 <= kOffMisc, "proxy rows must fit in the K/V ring");
-
-constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, 64, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, 128, true);
+// Shared-memory and MMA geometry for head dimension D.  A row of D bf16 channels is split into
+// D/64 swizzle atoms ("halves") of 64 channels = 128 bytes, each its own TMA box and buffer.
+template <int D>
+struct Geo {
+    static_assert(D == 64 || D == 128, "head dimension 64 or 128");
+    static constexpr int kHalves = D / 64;
+    static constexpr uint32_t kQBytes = kHalves * kQHalfBytes;
+    static constexpr uint32_t kKVTileBytes = kHalves * kKVHalfBytes;
+    static constexpr uint32_t kOffQ = 0;
+    static constexpr uint32_t kOffK = kOffQ + kQBytes;
+    static constexpr uint32_t kOffV = kOffK + kStages * kKVTileBytes;
+    static constexpr uint32_t kRingEnd = kOffV + kStages * kKVTileBytes;
+    static constexpr uint32_t kOffRowA = kOffK;          // proxy rows alias the K/V ring
+    static constexpr uint32_t kOffRowB = kOffK + kMaxBlocks * 4;
+    static constexpr uint32_t kRowsEnd = kOffRowB + kMaxBlocks * 4;
+    static constexpr uint32_t kOffMisc = ((kRingEnd > kRowsEnd ? kRingEnd : kRowsEnd) + 1023u) & ~1023u;
+    static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, 64, false);
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
+    static constexpr int kOChunks = D / 32;              // 32-column TMEM loads of a row of O
+    static constexpr int kLaneCh = D / 32;               // channels per lane in the proxy dot products
+    static_assert(kOffMisc % 1024 == 0, "shared-memory tiles need 1024-byte alignment");
+    static_assert(kTmemO + D <= kTmemCols, "O accumulator must fit in the TMEM allocation");
+};
 
 enum WaitSite : int {
     kSiteQ = 1, kSiteProdK = 2, kSiteProdV = 3, kSiteMmaK = 4, kSiteMmaP = 5, kSiteMmaV = 6,
@@ -101,16 +113,16 @@ struct Misc {
     uint32_t mask_b[kMaskWords];
     uint32_t mask_u[kMaskWords];
     uint32_t need[kChunkWords];
-    alignas(16) float qbar[2][kHeadDim];   // read as float4
+    alignas(16) float qbar[2][kMaxHeadDim];   // read as float4 / float2
     uint32_t tmem_base;
     int abort_flag;
     int count_a, count_b;
 };
 
-constexpr uint32_t kSmemBytes = kOffMisc + sizeof(Misc) + 1024;   // + alignment slack
+template <int D>
+constexpr uint32_t smem_bytes() { return Geo<D>::kOffMisc + sizeof(Misc) + 1024; }   // + alignment slack
 static_assert(offsetof(Misc, qbar) % 16 == 0, "q_bar is read with 16-byte vector loads");
 static_assert(offsetof(Misc, q_full) % 8 == 0, "mbarriers need 8-byte alignment");
-static_assert(kOffMisc % 1024 == 0, "shared-memory tiles need 1024-byte alignment");
 
 struct Params {
     int BH, N, Nk, Nq, npairs, nchunks;
@@ -196,11 +208,12 @@ __device__ __forceinline__ float bf16_at(const uint8_t *p)
 
 // ----------------------------------------------------------------------------- roles
 
+template <int D>
 __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int row, int bh)
 {
-    mbar_arrive_expect_tx(bar, kKVTileBytes);
-    tma_load_3d(dst, map, bar, 0, row, bh);
-    tma_load_3d(dst + kKVHalfBytes, map, bar, 64, row, bh);
+    mbar_arrive_expect_tx(bar, Geo<D>::kKVTileBytes);
+#pragma unroll
+    for (int h = 0; h < Geo<D>::kHalves; ++h) tma_load_3d(dst + h * kKVHalfBytes, map, bar, 64 * h, row, bh);
 }
 
 // One thread feeds both rings.  The tensor core retires work in the order
@@ -210,10 +223,12 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, 
 // stage that frees later.  K stage s is free when the QK of item it-2 has completed, which is the
 // phase of s_full[s] for that item (the S buffer and the K stage share the index); that phase
 // cannot be overtaken because QK(it) needs the tile loaded here.
+template <int D>
 __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                               const CUtensorMap *tm_kb, const CUtensorMap *tm_vb, uint8_t *smem,
                               Misc &m, const Params &p, int bh)
 {
+    using G = Geo<D>;
     int issued_k[kStages], issued_v[kStages];
     for (int s = 0; s < kStages; ++s) issued_k[s] = issued_v[s] = -1;
     Walker wk, wv;
@@ -223,7 +238,7 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
         if (more_k) {
             const int s = it & 1;
             if (it >= 2 && !wait_bar(&m.s_full[s], ((it - 2) >> 1) & 1, m, p, kSiteProdK)) { ok = false; break; }
-            load_tile(smem + kOffK + s * kKVTileBytes, wk.phase == 0 ? tm_kb : tm_k, &m.k_full[s], wk.idx * kTile, bh);
+            load_tile<D>(smem + G::kOffK + s * G::kKVTileBytes, wk.phase == 0 ? tm_kb : tm_k, &m.k_full[s], wk.idx * kTile, bh);
             issued_k[s] = it;
             more_k = wk.next(m, p);
         }
@@ -231,7 +246,7 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
         if (iv >= 0 && more_v) {
             const int s = iv & 1;
             if (iv >= 2 && !wait_bar(&m.v_empty[s], ((iv - 2) >> 1) & 1, m, p, kSiteProdV)) { ok = false; break; }
-            load_tile(smem + kOffV + s * kKVTileBytes, wv.phase == 0 ? tm_vb : tm_v, &m.v_full[s], wv.idx * kTile, bh);
+            load_tile<D>(smem + G::kOffV + s * G::kKVTileBytes, wv.phase == 0 ? tm_vb : tm_v, &m.v_full[s], wv.idx * kTile, bh);
             issued_v[s] = iv;
             more_v = wv.next(m, p);
         }
@@ -243,29 +258,33 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
     }
 }
 
+template <int D>
 __device__ __forceinline__ bool issue_pv(int t, uint32_t tmem, uint64_t dv0, Misc &m, const Params &p)
 {
+    using G = Geo<D>;
     const int b = t & 1, s = t & 1;
     const uint32_t ph = (t >> 1) & 1;
     if (!wait_bar(&m.p_full[b], ph, m, p, kSiteMmaP)) return false;
     if (!wait_bar(&m.v_full[s], ph, m, p, kSiteMmaV)) return false;
     tc_fence_after();
     // B = V tile of stage s, MN-major: 64 channels contiguous per key row (128 B, swizzled), next
-    // 8 keys at +1024 B (SBO), channels 64..127 at +8192 B (LBO); 16 keys per MMA -> +2048 B,
-    // i.e. +128 in the descriptor's 16-byte address units.
-    const uint64_t dv = dv0 + static_cast<uint64_t>(s) * (kKVTileBytes >> 4);
+    // 8 keys at +1024 B (SBO), channels 64..127 (d = 128) at +8192 B (LBO); 16 keys per MMA ->
+    // +2048 B, i.e. +128 in the descriptor's 16-byte address units.
+    const uint64_t dv = dv0 + static_cast<uint64_t>(s) * (G::kKVTileBytes >> 4);
     const uint32_t a0 = tmem + tmem_s_col(b);
-    if (t > 0) mma_ts_acc(tmem + kTmemO, a0, dv, kIdescPV);
-    else mma_ts(tmem + kTmemO, a0, dv, kIdescPV, 0u);
-    mma_ts_acc(tmem + kTmemO, a0 + 8, dv + 128, kIdescPV);
-    mma_ts_acc(tmem + kTmemO, a0 + 16, dv + 256, kIdescPV);
-    mma_ts_acc(tmem + kTmemO, a0 + 24, dv + 384, kIdescPV);
+    if (t > 0) mma_ts_acc(tmem + kTmemO, a0, dv, G::kIdescPV);
+    else mma_ts(tmem + kTmemO, a0, dv, G::kIdescPV, 0u);
+    mma_ts_acc(tmem + kTmemO, a0 + 8, dv + 128, G::kIdescPV);
+    mma_ts_acc(tmem + kTmemO, a0 + 16, dv + 256, G::kIdescPV);
+    mma_ts_acc(tmem + kTmemO, a0 + 24, dv + 384, G::kIdescPV);
     mma_commit(&m.v_empty[s]);
     return true;
 }
 
+template <int D>
 __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
 {
+    using G = Geo<D>;
     bool ok = true;
     if (p.fault_flags & 1) ok = wait_bar(&m.never, 0, m, p, kSiteFault);
     if (ok) ok = wait_bar(&m.q_full, 0, m, p, kSiteQ);
@@ -273,12 +292,12 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
         tc_fence_after();
         // Descriptors are built once; a k-step or stage only adds a compile-time offset to the
         // 14-bit start-address field (16-byte units; every address stays below 256 KB).
-        // A = Q (128 x 128), B = K tile (64 x 128), both K-major 128B-swizzled with 8-row groups
-        // 1024 B apart; channels 64..127 live in the second half buffer and a 16-channel step
-        // advances the start address by 32 B inside the swizzle atom.
-        const uint64_t dq = desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
-        const uint64_t dk0 = desc_sw128(smem_u32(smem + kOffK), 16, 1024);
-        const uint64_t dv0 = desc_sw128(smem_u32(smem + kOffV), kKVHalfBytes, 1024);
+        // A = Q (128 x d), B = K tile (64 x d), both K-major 128B-swizzled with 8-row groups
+        // 1024 B apart; channels 64..127 (d = 128) live in the second half buffer and a
+        // 16-channel step advances the start address by 32 B inside the swizzle atom.
+        const uint64_t dq = desc_sw128(smem_u32(smem + G::kOffQ), 16, 1024);
+        const uint64_t dk0 = desc_sw128(smem_u32(smem + G::kOffK), 16, 1024);
+        const uint64_t dv0 = desc_sw128(smem_u32(smem + G::kOffV), kKVHalfBytes, 1024);
         constexpr uint64_t kQh = kQHalfBytes >> 4, kKh = kKVHalfBytes >> 4;
         Walker w;
         int it = 0;
@@ -286,21 +305,23 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
             const int s = it & 1, b = it & 1;
             if (!wait_bar(&m.k_full[s], (it >> 1) & 1, m, p, kSiteMmaK)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t dk = dk0 + static_cast<uint64_t>(s) * (kKVTileBytes >> 4);
+            const uint64_t dk = dk0 + static_cast<uint64_t>(s) * (G::kKVTileBytes >> 4);
             const uint32_t d = tmem + tmem_s_col(b);
-            mma_ss(d, dq, dk, kIdescQK, 0u);
-            mma_ss_acc(d, dq + 2, dk + 2, kIdescQK);
-            mma_ss_acc(d, dq + 4, dk + 4, kIdescQK);
-            mma_ss_acc(d, dq + 6, dk + 6, kIdescQK);
-            mma_ss_acc(d, dq + kQh, dk + kKh, kIdescQK);
-            mma_ss_acc(d, dq + kQh + 2, dk + kKh + 2, kIdescQK);
-            mma_ss_acc(d, dq + kQh + 4, dk + kKh + 4, kIdescQK);
-            mma_ss_acc(d, dq + kQh + 6, dk + kKh + 6, kIdescQK);
+            mma_ss(d, dq, dk, G::kIdescQK, 0u);
+            mma_ss_acc(d, dq + 2, dk + 2, G::kIdescQK);
+            mma_ss_acc(d, dq + 4, dk + 4, G::kIdescQK);
+            mma_ss_acc(d, dq + 6, dk + 6, G::kIdescQK);
+            if constexpr (G::kHalves == 2) {
+                mma_ss_acc(d, dq + kQh, dk + kKh, G::kIdescQK);
+                mma_ss_acc(d, dq + kQh + 2, dk + kKh + 2, G::kIdescQK);
+                mma_ss_acc(d, dq + kQh + 4, dk + kKh + 4, G::kIdescQK);
+                mma_ss_acc(d, dq + kQh + 6, dk + kKh + 6, G::kIdescQK);
+            }
             mma_commit(&m.s_full[b]);
-            if (it > 0 && !issue_pv(it - 1, tmem, dv0, m, p)) { ok = false; break; }
+            if (it > 0 && !issue_pv<D>(it - 1, tmem, dv0, m, p)) { ok = false; break; }
             ++it;
         }
-        if (ok && it > 0 && issue_pv(it - 1, tmem, dv0, m, p)) mma_commit(&m.o_final);
+        if (ok && it > 0 && issue_pv<D>(it - 1, tmem, dv0, m, p)) mma_commit(&m.o_final);
     }
     // Every MMA issued so far must finish before TMEM is freed.
     mma_commit(&m.drain);
@@ -308,6 +329,7 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
 }
 
 // Softmax warps 0-3: thread r owns row r of the 128-row tile (TMEM lane r).
+template <int D>
 __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, int row0)
 {
     const int row = threadIdx.x;                       // 0..127 == TMEM lane
@@ -413,7 +435,7 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
             tc_fence_after();
             const float f = rescale ? factor : 1.0f;
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
                 uint32_t o[32];
                 const uint32_t oaddr = tmem + lane_base + kTmemO + ch * 32;
                 tmem_ld32(oaddr, o);
@@ -440,9 +462,9 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
     const int grow = row0 + row;
     const bool store = grow < p.N;
     const float inv_l = 1.0f / l;
-    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + (store ? grow : 0)) * kHeadDim);
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + (store ? grow : 0)) * D);
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + kTmemO + ch * 32, o);
         tmem_wait_ld();
@@ -462,14 +484,30 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
 
 // ----------------------------------------------------------------------------- kernel
 
+// Vector of LC consecutive floats loaded with one 8- or 16-byte access.
+template <int LC>
+__device__ __forceinline__ void load_vec(const float *src, float (&x)[LC])
+{
+    if constexpr (LC == 4) {
+        const float4 t = __ldg(reinterpret_cast<const float4 *>(src));
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    } else {
+        static_assert(LC == 2, "2 or 4 channels per lane");
+        const float2 t = __ldg(reinterpret_cast<const float2 *>(src));
+        x[0] = t.x; x[1] = t.y;
+    }
+}
+
+template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
                const __grid_constant__ CUtensorMap tm_vb, const Params p)
 {
+    using G = Geo<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Misc &m = *reinterpret_cast<Misc *>(smem + kOffMisc);
+    Misc &m = *reinterpret_cast<Misc *>(smem + G::kOffMisc);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pair = blockIdx.x % p.npairs;
     const int bh = blockIdx.x / p.npairs;
@@ -522,16 +560,17 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tmem = m.tmem_base;
 
     if (warp == kWarpTma && lane == 0) {
-        mbar_arrive_expect_tx(&m.q_full, kQBytes);
-        tma_load_3d(smem + kOffQ, &tm_q, &m.q_full, 0, row0, bh);
-        tma_load_3d(smem + kOffQ + kQHalfBytes, &tm_q, &m.q_full, 64, row0, bh);
+        mbar_arrive_expect_tx(&m.q_full, G::kQBytes);
+#pragma unroll
+        for (int h = 0; h < G::kHalves; ++h)
+            tma_load_3d(smem + G::kOffQ + h * kQHalfBytes, &tm_q, &m.q_full, 64 * h, row0, bh);
     }
 
     // ---------------- routing 1: q_bar of both routing tiles (float32, ascending rows)
-    if (tid < kHeadDim) {
+    if (tid < D) {
         if (wait_bar(&m.q_full, 0, m, p, kSiteQ)) {
             const int c = tid, half = c >> 6, cc = c & 63, chunk = cc >> 3, within = cc & 7;
-            const uint8_t *qh = smem + kOffQ + half * kQHalfBytes + within * 2;
+            const uint8_t *qh = smem + G::kOffQ + half * kQHalfBytes + within * 2;
             float sa = 0.0f, sb = 0.0f;
             for (int r = 0; r < n_a; ++r) sa += bf16_at(qh + r * 128 + ((chunk ^ (r & 7)) << 4));
             for (int r = 0; r < n_b; ++r) {
@@ -545,45 +584,56 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
 
     // ---------------- routing 2: proxy rows S_j = (q_bar . k_bar_j) * (1/sqrt d)
-    float *row_a = reinterpret_cast<float *>(smem + kOffRowA);
-    float *row_b = reinterpret_cast<float *>(smem + kOffRowB);
+    float *row_a = reinterpret_cast<float *>(smem + G::kOffRowA);
+    float *row_b = reinterpret_cast<float *>(smem + G::kOffRowB);
     const size_t unit_a = static_cast<size_t>(bh) * p.Nq + tile_a;
     {
         // Each warp takes groups of 8 key blocks (group g = blocks 8g..8g+7; warp w takes groups
-        // w, w+6, ...).  Lane l holds channels 4l..4l+3: it forms 16 partial dot products (8 blocks
-        // x tiles A/B) and a reduce-scatter over the lanes (16 shuffles) leaves the full sum of
-        // value (l >> 1) & 15 in lanes l and l^1.  The next group's rows are loaded before the
-        // current group is reduced.
-        const float4 qa = reinterpret_cast<const float4 *>(m.qbar[0])[lane];
-        const float4 qb = reinterpret_cast<const float4 *>(m.qbar[1])[lane];
-        const float4 *kb = reinterpret_cast<const float4 *>(p.kbar32 + static_cast<size_t>(bh) * Nk * kHeadDim) + lane;
+        // w, w+6, ...).  Lane l holds channels LC*l..LC*l+LC-1 (LC = d/32): it forms 16 partial
+        // dot products (8 blocks x tiles A/B) and a reduce-scatter over the lanes (16 shuffles)
+        // leaves the full sum of value (l >> 1) & 15 in lanes l and l^1.  The next group's rows are
+        // loaded before the current group is reduced.
+        constexpr int LC = G::kLaneCh;
+        float qa[LC], qb[LC];
+#pragma unroll
+        for (int c = 0; c < LC; ++c) {
+            qa[c] = m.qbar[0][LC * lane + c];
+            qb[c] = m.qbar[1][LC * lane + c];
+        }
+        const float *kb = p.kbar32 + static_cast<size_t>(bh) * Nk * D + LC * lane;
         const int ngroups = (Nk + 7) >> 3;
         const int my_idx = (lane >> 1) & 15;
         double sum_a = 0.0, sum_b = 0.0;
-        float4 x[8];
-        int g = warp;
-        if (g < ngroups) {
+        float x[8][LC];
+        auto load_group = [&](int grp) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int j = 8 * g + u;
-                x[u] = j < Nk ? __ldg(kb + static_cast<size_t>(j) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int j = 8 * grp + u;
+                if (j < Nk) {
+                    load_vec<LC>(kb + static_cast<size_t>(j) * D, x[u]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < LC; ++c) x[u][c] = 0.0f;
+                }
             }
-        }
+        };
+        int g = warp;
+        if (g < ngroups) load_group(g);
         for (; g < ngroups; g += kNumWarps) {
             float v[16];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                v[u] = fmaf(qa.w, x[u].w, fmaf(qa.z, x[u].z, fmaf(qa.y, x[u].y, qa.x * x[u].x)));
-                v[8 + u] = fmaf(qb.w, x[u].w, fmaf(qb.z, x[u].z, fmaf(qb.y, x[u].y, qb.x * x[u].x)));
+                float da = qa[0] * x[u][0], db = qb[0] * x[u][0];
+#pragma unroll
+                for (int c = 1; c < LC; ++c) {
+                    da = fmaf(qa[c], x[u][c], da);
+                    db = fmaf(qb[c], x[u][c], db);
+                }
+                v[u] = da;
+                v[8 + u] = db;
             }
             const int gn = g + kNumWarps;
-            if (gn < ngroups) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = 8 * gn + u;
-                    x[u] = j < Nk ? __ldg(kb + static_cast<size_t>(j) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
+            if (gn < ngroups) load_group(gn);
             float k8[8], k4[4], k2[2];
             const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4, h2 = lane & 2;
 #pragma unroll
@@ -735,15 +785,15 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const bool aborted = volatile_load(&m.abort_flag) != 0;
     if (warp == kWarpTma) {
         if (lane == 0) {
-            if (!aborted) producer_role(&tm_k, &tm_v, &tm_kb, &tm_vb, smem, m, p, bh);
+            if (!aborted) producer_role<D>(&tm_k, &tm_v, &tm_kb, &tm_vb, smem, m, p, bh);
             wait_bar(&m.q_full, 0, m, p, kSiteProdDrain, false);   // the Q copy has landed
         }
         __syncwarp();
     } else if (warp == kWarpMma) {
-        if (lane == 0 && !aborted) mma_role(tmem, smem, m, p);
+        if (lane == 0 && !aborted) mma_role<D>(tmem, smem, m, p);
         __syncwarp();
     } else if (!aborted) {
-        softmax_role(tmem, m, p, bh, row0);
+        softmax_role<D>(tmem, m, p, bh, row0);
     }
     tc_fence_before();
     __syncthreads();
@@ -753,19 +803,19 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-}  // namespace
-
-cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
+template <int D>
+cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
 {
     static std::once_flag attr_once[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    constexpr uint32_t kSmem = smem_bytes<D>();
     cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once[dev], [&] {
-        attr_err = cudaFuncSetAttribute(sol_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(kSmemBytes));
+        attr_err = cudaFuncSetAttribute(sol_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kSmem));
     });
     if (attr_err != cudaSuccess) return attr_err;
 
@@ -778,8 +828,8 @@ cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
     p.nchunks = (L.Nk + 63) / 64;
     p.beta = L.beta;
     p.beta_head = L.beta_head;
-    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
-    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     const int n_last = L.N - (L.Nk - 1) * kTile;
     p.last_bias_log2 = static_cast<float>(std::log2(static_cast<double>(n_last)));
     p.kbar32 = L.kbar32;
@@ -793,9 +843,18 @@ cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
     p.timeout_ns = L.timeout_ns;
     const long long grid = static_cast<long long>(p.npairs) * L.BH;
     if (grid <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    sol_fwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
+    sol_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(
         *L.tm_q, *L.tm_k, *L.tm_v, *L.tm_kb, *L.tm_vb, p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
+{
+    if (L.d == 128) return launch_d<128>(L, stream);
+    if (L.d == 64) return launch_d<64>(L, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace sol

@@ -162,12 +162,13 @@ def random_bf16(shape, seed: int, scale: float = 1.0) -> np.ndarray:
     return f32_to_bf16_bits(scale * rng.standard_normal(shape, dtype=np.float32))
 
 
-def small_workload(N: int, BH: int = 2, seed: int = 7, grid=None, f_max: float = 1.5):
-    """A small field+noise case with arbitrary (possibly ragged) N, shape [1, BH, N, 128]."""
+def small_workload(N: int, BH: int = 2, seed: int = 7, grid=None, f_max: float = 1.5,
+                   d: int = HEAD_DIM):
+    """A small field+noise case with arbitrary (possibly ragged) N, shape [1, BH, N, d]."""
     if grid is None:
         W = 32
         Hg = 16
         T = max(1, -(-N // (W * Hg)))
         grid = (T, Hg, W)
-    wl = Workload(f"small{N}", 1, BH, int(np.prod(grid)), tuple(grid), (), seed=seed, f_max=f_max)
+    wl = Workload(f"small{N}", 1, BH, int(np.prod(grid)), tuple(grid), (), seed=seed, f_max=f_max, d=d)
     return gen_workload(wl, n_tokens=N, processes=1)

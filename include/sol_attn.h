@@ -21,7 +21,8 @@
  *
  * Conventions for every entry point:
  *   - q, k, v, out: bfloat16, contiguous [B, H, N, d] (token rows of d elements), device
- *     pointers, 16-byte aligned.  d must be 128.  1 <= N <= 524288.  B*H*ceil(Nq/2) < 2^31.
+ *     pointers, 16-byte aligned.  d is 64 or 128 (the video DiT head sizes; the paper's models
+ *     use 128).  1 <= N <= 524288.  B*H*ceil(Nq/2) < 2^31.
  *   - The caller owns all memory.  The library allocates no device or host memory.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and
  *     stream-ordered.  sol_attn_fwd needs a prior sol_attn_pool on the same K, V and workspace,
@@ -46,7 +47,7 @@ extern "C" {
 typedef enum {
     SOL_OK = 0,
     SOL_ERR_INVALID_ARG = 1, /* null pointer, non-positive or too large size, NaN beta */
-    SOL_ERR_UNSUPPORTED = 2, /* d != 128, N above the supported maximum */
+    SOL_ERR_UNSUPPORTED = 2, /* d not 64 or 128, N above the supported maximum */
     SOL_ERR_ALIGNMENT = 3,   /* a tensor pointer that is not 16-byte aligned */
     SOL_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
     SOL_ERR_TIMEOUT = 5,     /* a device pipeline wait gave up (see sol_attn_read_status) */
@@ -125,8 +126,8 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
  * the pooled keys/values and status words go to a scratch array inside the library instead of a
  * caller workspace.  This entry point calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Limit: sol_attn_workspace_bytes(B, H, N, d) <= SOL_ATTN_NOALLOC_MAX_BYTES, i.e.
- *     B*H*ceil(N/64) <= 10922 pooled rows (a 12-head, 16384-token call fits); larger shapes
- *     return SOL_ERR_SCRATCH_LIMIT without launching anything.
+ *     B*H*ceil(N/64) <= 10922 pooled rows at d = 128, 21845 at d = 64 (a 12-head, 16384-token
+ *     call fits); larger shapes return SOL_ERR_SCRATCH_LIMIT without launching anything.
  *   - The first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any stream
  *     capture.

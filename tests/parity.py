@@ -46,7 +46,7 @@ def gpu_run(q, k, v, beta: float, debug: bool = True, units=None, with_proxy: bo
     assert st == 0, (sol.STATUS.get(st), where)
     sel = None if units is None else torch.as_tensor(np.asarray(units), device="cuda")
     pick = (lambda t: t.reshape(B * H * Nq, *t.shape[3:]).index_select(0, sel)) if sel is not None else (lambda t: t)
-    kb32 = sol.workspace_views(ws, B, H, N)[0]
+    kb32 = sol.workspace_views(ws, B, H, N, d)[0]
     res = dict(density=dens.cpu().numpy(), units=units, kbar32=kb32.cpu().numpy())
     if sel is None:
         res["out"] = out.float().cpu().numpy()

@@ -44,7 +44,13 @@ def test_workspace_bytes(lib):
     got = sol.sol_attn_workspace_bytes(B, H, N, 128)
     assert got >= 256 + n * (4 + 4 + 2 + 2) and got % 256 == 0
     assert sol.sol_attn_workspace_bytes(1, 1, 100, 128) > 0
-    assert sol.sol_attn_workspace_bytes(1, 1, 100, 64) == 0       # d != 128 unsupported
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 96) == 0       # d not 64/128: unsupported
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 256) == 0
+    # d = 64: the same layout with 64-channel rows
+    Nk64 = 2
+    n64 = 1 * 1 * Nk64 * 64
+    up = lambda x: (x + 255) & ~255
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 64) == up(up(up(up(256 + 4 * n64) + 4 * n64) + 2 * n64) + 2 * n64)
     assert sol.sol_attn_workspace_bytes(0, 1, 100, 128) == 0
     assert sol.sol_attn_workspace_bytes(1, 1, 524288 + 1, 128) == 0
 
@@ -65,7 +71,7 @@ def fwd(lib, q=A, k=A, v=A, B=1, H=1, N=128, d=128, beta=0.5, ws=A, out=A, dens=
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(q=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
-    (dict(N=0), 1), (dict(B=-1), 1), (dict(d=64), 2), (dict(N=524288 + 64), 2),
+    (dict(N=0), 1), (dict(B=-1), 1), (dict(d=96), 2), (dict(d=256), 2), (dict(N=524288 + 64), 2),
     (dict(beta=math.nan), 1), (dict(k=MIS), 3), (dict(ws=A + 16), 3), (dict(dens=A + 2), 3),
 ])
 def test_fwd_rejects_bad_arguments_on_host(lib, kw, expect):

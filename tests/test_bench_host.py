@@ -27,6 +27,12 @@ def test_flop_counts_hand_computed():
     # tile pairs (0,1) and (2,3): unions of 4 and 1 kept blocks; one correction chunk each
     # (tile 0 and tile 2 skip blocks) -> 7 MMA iterations of 128 x 64 keys
     assert fc["executed"] == 4 * 128 * 128 * 64 * (4 + 1 + 2)
+    # token-weighted density: computed (query, key) pairs over N^2
+    pairs = 64 * 64 + 16 * 16 + 64 * 208
+    assert abs(fc["density_tokens"] - pairs / 208 ** 2) < 1e-15
+    # d scales every flop count but no density
+    fc64 = bench.flop_counts(mask, N, d=64)
+    assert fc64["kept"] == kept / 2 and fc64["density_tokens"] == fc["density_tokens"]
 
 
 def test_replica_throughput():

@@ -12,16 +12,18 @@ from parity import to_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,H,N", [(1, 2, 4096), (2, 3, 64 * 9 + 16), (1, 1, 1), (1, 2, 63), (1, 4, 1000)])
-def test_pool_bit_exact(B, H, N):
-    k = inputs.random_bf16((B, H, N, 128), seed=N + 1, scale=3.0)
-    v = inputs.random_bf16((B, H, N, 128), seed=N + 2)
-    ws = torch.zeros(sol.sol_attn_workspace_bytes(B, H, N, 128), dtype=torch.uint8, device="cuda")
+@pytest.mark.parametrize("B,H,N,d", [(1, 2, 4096, 128), (2, 3, 64 * 9 + 16, 128), (1, 1, 1, 128),
+                                     (1, 2, 63, 128), (1, 4, 1000, 128), (1, 2, 4096, 64),
+                                     (2, 3, 64 * 9 + 16, 64), (1, 1, 1, 64), (1, 3, 1000, 64)])
+def test_pool_bit_exact(B, H, N, d):
+    k = inputs.random_bf16((B, H, N, d), seed=N + 1, scale=3.0)
+    v = inputs.random_bf16((B, H, N, d), seed=N + 2)
+    ws = torch.zeros(sol.sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
     sol.sol_attn_pool(to_dev(k), to_dev(v), ws)
     torch.cuda.synchronize()
-    k32, v32, k16, v16 = (t.cpu() for t in sol.workspace_views(ws, B, H, N))
+    k32, v32, k16, v16 = (t.cpu() for t in sol.workspace_views(ws, B, H, N, d))
     Nk = (N + 63) // 64
-    rk, rv = sol_ref.pool(k).reshape(B, H, Nk, 128), sol_ref.pool(v).reshape(B, H, Nk, 128)
+    rk, rv = sol_ref.pool(k).reshape(B, H, Nk, d), sol_ref.pool(v).reshape(B, H, Nk, d)
     assert np.array_equal(k32.numpy(), rk)
     assert np.array_equal(v32.numpy(), rv)
     assert np.array_equal(k16.view(torch.int16).numpy().view(np.uint16), inputs.f32_to_bf16_bits(rk))

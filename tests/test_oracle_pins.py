@@ -69,19 +69,20 @@ def test_pool_ragged_block_divides_by_its_own_length():
 
 # ---------------------------------------------------------------- attention limits
 
-def _head(N, seed=3, BH=2):
-    q, k, v = inputs.small_workload(N, BH=BH, seed=seed)
+def _head(N, seed=3, BH=2, d=D):
+    q, k, v = inputs.small_workload(N, BH=BH, seed=seed, d=d)
     return q[0], k[0], v[0]
 
 
-@pytest.mark.parametrize("N", [200, 64 * 3])
-def test_dense_limit_equals_sdpa(N):
-    """beta = -inf keeps every block: plain dense softmax attention."""
-    q, k, v = _head(N)
+@pytest.mark.parametrize("N,d", [(200, D), (64 * 3, D), (200, 64)])
+def test_dense_limit_equals_sdpa(N, d):
+    """beta = -inf keeps every block: plain dense softmax attention (scale 1/sqrt(d) from the
+    library routine, so a hard-wired head size fails at d = 64)."""
+    q, k, v = _head(N, d=d)
     r = sol_ref.forward(q, k, v, float("-inf"))
     Nk = (N + T - 1) // T
     assert np.all(r["count"] == Nk)
-    out = r["out"].reshape(2, Nk, T, D)
+    out = r["out"].reshape(2, Nk, T, d)
     for bh in range(2):
         want = sdpa64(f32(q[bh]), f32(k[bh]), f32(v[bh]))
         np.testing.assert_allclose(all_rows(out[bh], N), want, rtol=0, atol=1e-10)
@@ -94,14 +95,15 @@ def test_large_beta_keeps_no_block(beta):
     assert r["count"].sum() == 0 and r["mask"].sum() == 0
 
 
-def test_zero_selection_equals_dense_over_pooled_sequence():
+@pytest.mark.parametrize("d", [D, 64])
+def test_zero_selection_equals_dense_over_pooled_sequence(d):
     """With nothing kept, each block j acts as n_j copies of (k_bar_j, v_bar_j)."""
     N = 64 * 5 + 16
-    q, k, v = _head(N, seed=11)
+    q, k, v = _head(N, seed=11, d=d)
     r = sol_ref.forward(q, k, v, float("inf"))
     Nk = (N + T - 1) // T
     lens = [min(N, (j + 1) * T) - j * T for j in range(Nk)]
-    out = r["out"].reshape(2, Nk, T, D)
+    out = r["out"].reshape(2, Nk, T, d)
     for bh in range(2):
         kk = np.repeat(r["kbar"][bh].astype(np.float64), lens, axis=0)
         vv = np.repeat(r["vbar"][bh].astype(np.float64), lens, axis=0)
@@ -228,10 +230,10 @@ def test_two_blocks_have_unit_z_scores(seed):
 
 # ---------------------------------------------------------------- routing vs library statistics
 
-@pytest.mark.parametrize("beta", [0.0, 0.7, 1.3, -0.4])
-def test_routing_matches_numpy_statistics(beta):
+@pytest.mark.parametrize("beta,d", [(0.0, D), (0.7, D), (1.3, D), (-0.4, D), (0.7, 64)])
+def test_routing_matches_numpy_statistics(beta, d):
     N = 64 * 40 + 16
-    q, k, _ = _head(N, seed=9)
+    q, k, _ = _head(N, seed=9, d=d)
     Nk = (N + T - 1) // T
     r = sol_ref.route(q, sol_ref.pool(k), beta)
     qf, kf = f32(q).astype(np.float64), f32(k).astype(np.float64)
@@ -239,7 +241,7 @@ def test_routing_matches_numpy_statistics(beta):
     for bh in range(2):
         qb = np.stack([qf[bh, j * T:(j + 1) * T].mean(0) for j in range(Nk)])
         kb = np.stack([kf[bh, j * T:(j + 1) * T].mean(0) for j in range(Nk)])
-        S = qb @ kb.T / math.sqrt(D)
+        S = qb @ kb.T / math.sqrt(d)
         mu, sd = S.mean(1), S.std(1)
         tau = mu + beta * sd
         sl = slice(bh * Nk, (bh + 1) * Nk)
