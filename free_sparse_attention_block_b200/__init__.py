@@ -21,6 +21,7 @@ __all__ = [
     "sol_attn_workspace_bytes", "sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug",
     "sol_attn_read_status", "sol_attn_fwd_host", "sol_attn_error_string", "forward",
     "workspace_views", "sol_attn_fwd_noalloc", "NOALLOC_MAX_BYTES", "sol_attn_fwd_betas",
+    "sol_attn_fwd_topk", "sol_attn_fwd_topp", "sol_attn_fwd_debug_route", "ROUTE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
@@ -30,6 +31,7 @@ TILE = 64
 STATUS = {0: "SOL_OK", 1: "SOL_ERR_INVALID_ARG", 2: "SOL_ERR_UNSUPPORTED", 3: "SOL_ERR_ALIGNMENT",
           4: "SOL_ERR_CUDA", 5: "SOL_ERR_TIMEOUT", 6: "SOL_ERR_SCRATCH_LIMIT"}
 NOALLOC_MAX_BYTES = 16 * 1024 * 1024
+ROUTE = {"threshold": 0, "topk": 1, "topp": 2}     # sol_route
 
 _lock = threading.Lock()
 _lib = None
@@ -62,10 +64,14 @@ def load_library(path: str | None = None):
         lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.sol_attn_fwd_noalloc.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         lib.sol_attn_fwd_betas.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
+        lib.sol_attn_fwd_topk.argtypes = [vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp]
+        lib.sol_attn_fwd_topp.argtypes = [vp, vp, vp, i, i, i, i, f, vp, vp, vp, vp]
+        lib.sol_attn_fwd_debug_route.argtypes = [vp, vp, vp, i, i, i, i, i, f, vp, vp, vp, vp, vp, vp, vp]
         lib.sol_attn_error_string.argtypes = [i]
         lib.sol_attn_error_string.restype = C.c_char_p
         for name in ("sol_attn_pool", "sol_attn_fwd", "sol_attn_fwd_debug", "sol_attn_read_status",
-                     "sol_attn_fwd_host", "sol_attn_fwd_noalloc", "sol_attn_fwd_betas"):
+                     "sol_attn_fwd_host", "sol_attn_fwd_noalloc", "sol_attn_fwd_betas",
+                     "sol_attn_fwd_topk", "sol_attn_fwd_topp", "sol_attn_fwd_debug_route"):
             getattr(lib, name).restype = C.c_int
         if path is None:
             _lib = lib
@@ -139,6 +145,41 @@ def sol_attn_fwd_betas(q, k, v, beta_per_head, workspace, out, density_out=None,
     if check:
         _check(st, "sol_attn_fwd_betas")
     return st
+
+
+def sol_attn_fwd_topk(q, k, v, k_blocks: int, workspace, out, density_out=None, stream=None,
+                      check: bool = True) -> int:
+    """Forward with the top-k rule: the k_blocks highest-scoring blocks per query tile."""
+    B, H, N, d = _shape(q)
+    st = load_library().sol_attn_fwd_topk(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(k_blocks),
+                                          _ptr(workspace), _ptr(out), _ptr(density_out),
+                                          _stream(stream))
+    if check:
+        _check(st, "sol_attn_fwd_topk")
+    return st
+
+
+def sol_attn_fwd_topp(q, k, v, p: float, workspace, out, density_out=None, stream=None,
+                      check: bool = True) -> int:
+    """Forward with the top-p rule: the shortest highest-first prefix of blocks whose softmax
+    probability over the proxy row reaches p."""
+    B, H, N, d = _shape(q)
+    st = load_library().sol_attn_fwd_topp(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(p),
+                                          _ptr(workspace), _ptr(out), _ptr(density_out),
+                                          _stream(stream))
+    if check:
+        _check(st, "sol_attn_fwd_topp")
+    return st
+
+
+def sol_attn_fwd_debug_route(q, k, v, route, param: float, workspace, out, density_out=None,
+                             proxy_out=None, mask_out=None, stats_out=None, stream=None) -> int:
+    """Debug forward for any rule (``route``: a ROUTE name or code).  Returns the status code."""
+    B, H, N, d = _shape(q)
+    code = ROUTE[route] if isinstance(route, str) else int(route)
+    return load_library().sol_attn_fwd_debug_route(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, code, float(param), _ptr(workspace), _ptr(out),
+        _ptr(density_out), _ptr(proxy_out), _ptr(mask_out), _ptr(stats_out), _stream(stream))
 
 
 def sol_attn_fwd_debug(q, k, v, beta: float, workspace, out, density_out=None, proxy_out=None,

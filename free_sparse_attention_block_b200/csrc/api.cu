@@ -92,10 +92,17 @@ bool encode_rows(CUtensorMap *map, const void *base, long long rows, int BH, int
     return r == CUDA_SUCCESS;
 }
 
+// Routing rule and its parameter for one call.
+struct RouteArg {
+    int route = kRouteThreshold;
+    int topk = 0;
+    float topp = 0.0f;
+};
+
 sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
                    float beta, const float *beta_head, void *workspace, void *out, int32_t *density,
                    float *dbg_proxy, uint8_t *dbg_mask, float *dbg_stats, int fault_flags,
-                   unsigned long long timeout_ns, cudaStream_t stream)
+                   unsigned long long timeout_ns, cudaStream_t stream, RouteArg ra = RouteArg{})
 {
     Shape s{};
     sol_status st = check_shape(B, H, N, d, &s);
@@ -137,10 +144,33 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     L.dbg_stats = dbg_stats;
     L.fault_flags = fault_flags;
     L.timeout_ns = timeout_ns;
+    L.route = ra.route;
+    L.topk = ra.topk;
+    L.topp = ra.topp;
     return launch_sol_fwd(L, stream) == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
 }
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000ull * 1000ull * 1000ull;   // 2 s
+
+// Validates a rule and its parameter: top-k needs k >= 0 (values above Nk keep every block),
+// top-p a non-NaN p (<= 0 keeps none, >= 1 keeps every block).
+sol_status route_arg(int route, double param, RouteArg *ra)
+{
+    ra->route = route;
+    switch (route) {
+    case kRouteThreshold:
+        return std::isnan(param) ? SOL_ERR_INVALID_ARG : SOL_OK;
+    case kRouteTopK:
+        if (std::isnan(param) || param < 0.0 || param != std::floor(param)) return SOL_ERR_INVALID_ARG;
+        ra->topk = param > 1e9 ? 1000000000 : static_cast<int>(param);
+        return SOL_OK;
+    case kRouteTopP:
+        if (std::isnan(param)) return SOL_ERR_INVALID_ARG;
+        ra->topp = static_cast<float>(param);
+        return SOL_OK;
+    }
+    return SOL_ERR_INVALID_ARG;
+}
 
 }  // namespace
 }  // namespace sol
@@ -189,6 +219,46 @@ sol_status sol_attn_fwd_betas(const void *q, const void *k, const void *v, int B
     if (!beta_per_head) return SOL_ERR_INVALID_ARG;
     return run_fwd(q, k, v, B, H, N, d, 0.0f, beta_per_head, workspace, out, density_out, nullptr,
                    nullptr, nullptr, 0, kDefaultTimeoutNs, static_cast<cudaStream_t>(stream));
+}
+
+sol_status sol_attn_fwd_topk(const void *q, const void *k, const void *v, int B, int H, int N,
+                             int d, int k_blocks, void *workspace, void *out, int32_t *density_out,
+                             void *stream)
+{
+    RouteArg ra;
+    const sol_status st = route_arg(kRouteTopK, static_cast<double>(k_blocks), &ra);
+    if (st != SOL_OK) return st;
+    return run_fwd(q, k, v, B, H, N, d, 0.0f, nullptr, workspace, out, density_out, nullptr,
+                   nullptr, nullptr, 0, kDefaultTimeoutNs, static_cast<cudaStream_t>(stream), ra);
+}
+
+sol_status sol_attn_fwd_topp(const void *q, const void *k, const void *v, int B, int H, int N,
+                             int d, float p, void *workspace, void *out, int32_t *density_out,
+                             void *stream)
+{
+    RouteArg ra;
+    const sol_status st = route_arg(kRouteTopP, static_cast<double>(p), &ra);
+    if (st != SOL_OK) return st;
+    return run_fwd(q, k, v, B, H, N, d, 0.0f, nullptr, workspace, out, density_out, nullptr,
+                   nullptr, nullptr, 0, kDefaultTimeoutNs, static_cast<cudaStream_t>(stream), ra);
+}
+
+sol_status sol_attn_fwd_debug_route(const void *q, const void *k, const void *v, int B, int H,
+                                    int N, int d, int route, float param, void *workspace,
+                                    void *out, int32_t *density_out, float *proxy_out,
+                                    uint8_t *mask_out, float *stats_out, void *stream)
+{
+    if ((proxy_out && !aligned16(proxy_out)) || (stats_out && !aligned16(stats_out)))
+        return SOL_ERR_ALIGNMENT;
+    RouteArg ra;
+    sol_status st = route_arg(route, static_cast<double>(param), &ra);
+    if (st != SOL_OK) return st;
+    const float beta = route == kRouteThreshold ? param : 0.0f;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    st = run_fwd(q, k, v, B, H, N, d, beta, nullptr, workspace, out, density_out, proxy_out,
+                 mask_out, stats_out, 0, kDefaultTimeoutNs, cs, ra);
+    if (st != SOL_OK) return st;
+    return sol_attn_read_status(workspace, nullptr, stream);
 }
 
 sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream)

@@ -29,6 +29,11 @@ WorkspaceLayout workspace_layout(long long BH, long long Nk, int d);
 cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, int d, float *kbar32,
                            float *vbar32, void *kbar16, void *vbar16, cudaStream_t stream);
 
+// Block-selection rule of the routing step.  The page's own rule is the threshold
+// mu + beta*sigma; top-k and top-p are the prior-art rules it compares against, run on the same
+// proxy row in the same kernel.
+enum Route : int { kRouteThreshold = 0, kRouteTopK = 1, kRouteTopP = 2 };
+
 struct FwdLaunch {
     const CUtensorMap *tm_q, *tm_k, *tm_v, *tm_kb, *tm_vb;
     int BH, N, Nk, Nq, d;
@@ -43,6 +48,9 @@ struct FwdLaunch {
     float *dbg_stats;
     int fault_flags;
     unsigned long long timeout_ns;
+    int route;      // Route
+    int topk;       // kRouteTopK: blocks kept per query tile
+    float topp;     // kRouteTopP: probability mass covered per query tile
 };
 cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream);
 

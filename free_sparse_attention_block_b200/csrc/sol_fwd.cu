@@ -98,6 +98,8 @@ struct Geo {
     static_assert(kTmemO + D <= kTmemCols, "O accumulator must fit in the TMEM allocation");
 };
 
+enum SelState : int { kSelRun = 0, kSelNone = 1, kSelAll = 2 };
+
 enum WaitSite : int {
     kSiteQ = 1, kSiteProdK = 2, kSiteProdV = 3, kSiteMmaK = 4, kSiteMmaP = 5, kSiteMmaV = 6,
     kSiteSoftS = 7, kSiteSoftO = 8, kSiteEpilogue = 9, kSiteFault = 10, kSiteDrain = 11,
@@ -114,6 +116,16 @@ struct Misc {
     uint32_t mask_u[kMaskWords];
     uint32_t need[kChunkWords];
     alignas(16) float qbar[2][kMaxHeadDim];   // read as float4 / float2
+    // radix selection of the top-k / top-p routing rules; index 0 = tile A, 1 = tile B
+    double hist_mass[2][256];
+    uint32_t hist_cnt[2][256];
+    double sel_target[2];     // blocks (top-k) or probability mass (top-p) still to be covered
+    float row_max[2];
+    uint32_t sel_key[2];      // score key of the last kept block
+    uint32_t sel_min[2];      // smallest kept key (the threshold statistic of the debug output)
+    int sel_state[2];         // kSelRun, kSelNone or kSelAll
+    int sel_ceq[2];           // blocks whose key equals sel_key
+    int sel_neq[2];           // how many of those (lowest indices first) are kept
     uint32_t tmem_base;
     int abort_flag;
     int count_a, count_b;
@@ -121,6 +133,8 @@ struct Misc {
 
 template <int D>
 constexpr uint32_t smem_bytes() { return Geo<D>::kOffMisc + sizeof(Misc) + 1024; }   // + alignment slack
+// 228 KB of shared memory per SM, of which the driver reserves 1 KB per CTA
+static_assert(2 * (smem_bytes<128>() + 1024) <= 228 * 1024, "two CTAs must fit on an SM");
 static_assert(offsetof(Misc, qbar) % 16 == 0, "q_bar is read with 16-byte vector loads");
 static_assert(offsetof(Misc, q_full) % 8 == 0, "mbarriers need 8-byte alignment");
 
@@ -140,6 +154,9 @@ struct Params {
     float *dbg_stats;
     int fault_flags;
     unsigned long long timeout_ns;
+    int route;               // kRouteThreshold, kRouteTopK or kRouteTopP
+    int topk;                // blocks kept per query tile (top-k)
+    float topp;              // probability mass to cover per query tile (top-p)
 };
 
 __device__ __forceinline__ int volatile_load(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
@@ -485,6 +502,215 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
 // ----------------------------------------------------------------------------- kernel
 
 // Vector of LC consecutive floats loaded with one 8- or 16-byte access.
+// ----------------------------------------------------------------------------- top-k / top-p
+
+// Order-preserving 32-bit key of a score: a larger float gives a larger key; -0.0 and +0.0 (equal
+// scores) share the key of +0.0.
+__device__ __forceinline__ uint32_t score_key(float x)
+{
+    const uint32_t u = __float_as_uint(x == 0.0f ? 0.0f : x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_score(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Radix selection (four 8-bit digits, most significant first) of the last kept block of the
+// top-k or top-p rule, for both routing tiles at once; all threads of the CTA take part.
+// Blocks are ranked by score, highest first, equal scores by ascending index.  Top-k keeps the
+// first k; top-p keeps the shortest prefix whose softmax mass (float64, w_j = exp(S_j - max S))
+// reaches p * Z.  Each pass histograms the digit of the blocks whose higher digits equal the
+// selected prefix (counts, and for top-p masses) and one warp per tile walks the histogram from
+// the top bin down to the bin that holds the last kept block.  Result per tile t: sel_key[t] and
+// sel_neq[t] -- keep key > sel_key, and the first sel_neq[t] (by index) of the sel_ceq[t] blocks
+// whose key equals sel_key -- or sel_state[t] = kSelNone / kSelAll.
+__device__ void radix_select(const float *row_a, const float *row_b, bool has_b, int Nk, Misc &m,
+                             const Params &p)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool topp = p.route == kRouteTopP;
+    if (topp) {   // row maxima for the softmax masses
+        float ma = -INFINITY, mb = -INFINITY;
+        for (int j = tid; j < Nk; j += kThreads) {
+            ma = fmaxf(ma, row_a[j]);
+            mb = fmaxf(mb, row_b[j]);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            ma = fmaxf(ma, __shfl_xor_sync(0xFFFFFFFFu, ma, o));
+            mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+        }
+        if (lane == 0) {
+            m.red[0][warp] = ma;
+            m.red[1][warp] = mb;
+        }
+    }
+    __syncthreads();
+    if (tid < 2) {
+        const int t = tid;
+        if (topp) {
+            float mx = -INFINITY;
+            for (int w = 0; w < kNumWarps; ++w) mx = fmaxf(mx, static_cast<float>(m.red[t][w]));
+            m.row_max[t] = mx;
+        }
+        int state = kSelRun;
+        double target = 0.0;
+        if (t == 1 && !has_b) {
+            state = kSelNone;
+        } else if (topp) {
+            if (p.topp >= 1.0f) state = kSelAll;
+            else if (!(p.topp > 0.0f)) state = kSelNone;   // target p*Z is set in the first pass
+        } else {
+            const int need = min(p.topk, Nk);
+            if (need <= 0) state = kSelNone;
+            else if (need >= Nk) state = kSelAll;
+            target = need;
+        }
+        m.sel_state[t] = state;
+        m.sel_target[t] = target;
+        m.sel_key[t] = 0u;
+        m.sel_min[t] = 0xFFFFFFFFu;
+        m.sel_ceq[t] = 0;
+        m.sel_neq[t] = 0;
+    }
+    __syncthreads();
+    if (m.sel_state[0] != kSelRun && m.sel_state[1] != kSelRun) return;
+
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        for (int i = tid; i < 256; i += kThreads) {
+            m.hist_cnt[0][i] = 0u;
+            m.hist_cnt[1][i] = 0u;
+            m.hist_mass[0][i] = 0.0;
+            m.hist_mass[1][i] = 0.0;
+        }
+        __syncthreads();
+        for (int t = 0; t < 2; ++t) {
+            if (m.sel_state[t] != kSelRun) continue;
+            const float *row = t ? row_b : row_a;
+            const uint32_t pre = m.sel_key[t];
+            const double mx = m.row_max[t];
+            for (int j = tid; j < Nk; j += kThreads) {
+                const float sc = row[j];
+                const uint32_t key = score_key(sc);
+                if ((key ^ pre) & hi_mask) continue;
+                const int dig = (key >> shift) & 255;
+                atomicAdd(&m.hist_cnt[t][dig], 1u);
+                if (topp) atomicAdd(&m.hist_mass[t][dig], exp(static_cast<double>(sc) - mx));
+            }
+        }
+        __syncthreads();
+        if (warp < 2 && m.sel_state[warp] == kSelRun) {
+            const int t = warp;
+            // lane l holds bins 8l..8l+7; higher bins hold higher scores
+            double v[8];
+            uint32_t c[8];
+            double tot = 0.0;
+            uint32_t ctot = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = m.hist_cnt[t][8 * lane + i];
+                v[i] = topp ? m.hist_mass[t][8 * lane + i] : static_cast<double>(c[i]);
+                tot += v[i];
+                ctot += c[i];
+            }
+            double incl = tot;   // sum over lanes l..31
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double n = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+                if (lane + o < 32) incl += n;
+            }
+            double target = m.sel_target[t];
+            if (topp && pass == 0) target = static_cast<double>(p.topp) * __shfl_sync(0xFFFFFFFFu, incl, 0);
+            // the bin of the last kept block is in the highest lane whose suffix sum reaches the
+            // target; if rounding leaves every lane short, the lowest non-empty lane is used
+            const uint32_t reach = __ballot_sync(0xFFFFFFFFu, incl >= target);
+            const uint32_t nonempty = __ballot_sync(0xFFFFFFFFu, ctot != 0u);
+            const int sel_lane = reach ? 31 - __clz(reach) : __ffs(nonempty) - 1;
+            if (lane == sel_lane) {
+                double acc = incl - tot;          // mass/count of the higher lanes
+                // first bin (from the top) whose running sum reaches the target; if rounding
+                // leaves every bin just short, the lowest non-empty bin
+                int bin = -1, low = -1;
+                uint32_t cnt = 0u, low_cnt = 0u;
+                double before = acc, low_before = acc;
+#pragma unroll
+                for (int i = 7; i >= 0; --i) {
+                    if (bin >= 0 || c[i] == 0u) continue;
+                    if (acc + v[i] >= target) {
+                        bin = i;
+                        cnt = c[i];
+                        before = acc;
+                    } else {
+                        low = i;
+                        low_cnt = c[i];
+                        low_before = acc;
+                        acc += v[i];
+                    }
+                }
+                if (bin < 0) {
+                    bin = low;
+                    cnt = low_cnt;
+                    before = low_before;
+                }
+                m.sel_key[t] |= static_cast<uint32_t>(8 * lane + bin) << shift;
+                m.sel_target[t] = target - before;
+                m.sel_ceq[t] = static_cast<int>(cnt);
+            }
+        }
+        __syncthreads();
+    }
+    if (tid < 2 && m.sel_state[tid] == kSelRun) {
+        const int t = tid;
+        const int ceq = m.sel_ceq[t];
+        const double rem = m.sel_target[t];
+        int n;
+        if (topp) {
+            // blocks with the selected key have equal masses; add them in index order until the
+            // remaining mass is covered
+            const double w = exp(static_cast<double>(key_score(m.sel_key[t])) - static_cast<double>(m.row_max[t]));
+            double acc = 0.0;
+            n = 0;
+            while (n < ceq && acc < rem) {
+                acc += w;
+                ++n;
+            }
+            n = max(n, 1);
+        } else {
+            n = static_cast<int>(rem);
+        }
+        m.sel_neq[t] = min(max(n, 1), ceq);
+    }
+    __syncthreads();
+}
+
+// Keep decision of the top-k / top-p rules before ties at the selected key are thinned out.
+__device__ __forceinline__ bool sel_keep(const Misc &m, int t, uint32_t key)
+{
+    const int st = m.sel_state[t];
+    return st == kSelAll || (st == kSelRun && key >= m.sel_key[t]);
+}
+
+// Blocks whose key equals the selected key are all marked kept by sel_keep; keep only the first
+// sel_neq of them (by index).  One thread per tile; runs only when such ties exist.
+__device__ void thin_ties(uint32_t *mask, const float *row, int Nk, Misc &m, int t, int *count)
+{
+    if (m.sel_state[t] != kSelRun || m.sel_neq[t] >= m.sel_ceq[t]) return;
+    const uint32_t ks = m.sel_key[t];
+    int seen = 0;
+    for (int j = 0; j < Nk; ++j) {
+        if (score_key(row[j]) != ks) continue;
+        if (seen >= m.sel_neq[t]) {
+            mask[j >> 5] &= ~(1u << (j & 31));
+            --*count;
+        }
+        ++seen;
+    }
+}
+
 template <int LC>
 __device__ __forceinline__ void load_vec(const float *src, float (&x)[LC])
 {
@@ -722,17 +948,29 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncthreads();
     // ---------------- routing 4: keep masks (ballot per 32 blocks), counts, debug rows
+    const bool by_rank = p.route != kRouteThreshold;   // top-k / top-p instead of mu + beta*sigma
+    if (by_rank) radix_select(row_a, row_b, has_b, Nk, m, p);
+    const int nwords = (Nk + 31) >> 5;
     {
         const double tau_a = m.tau[0], tau_b = m.tau[1];
-        const int nwords = (Nk + 31) >> 5;
         int cnt_a = 0, cnt_b = 0;
+        uint32_t min_a = 0xFFFFFFFFu, min_b = 0xFFFFFFFFu;
         for (int wd = warp; wd < nwords; wd += kNumWarps) {
             const int j = wd * 32 + lane;
             const bool inb = j < Nk;
             const float sa = inb ? row_a[j] : 0.0f;
             const float sb = inb ? row_b[j] : 0.0f;
-            const bool ka = inb && static_cast<double>(sa) >= tau_a;
-            const bool kb = inb && has_b && static_cast<double>(sb) >= tau_b;
+            bool ka, kb;
+            if (by_rank) {
+                const uint32_t ya = score_key(sa), yb = score_key(sb);
+                ka = inb && sel_keep(m, 0, ya);
+                kb = inb && has_b && sel_keep(m, 1, yb);
+                if (ka) min_a = min(min_a, ya);
+                if (kb) min_b = min(min_b, yb);
+            } else {
+                ka = inb && static_cast<double>(sa) >= tau_a;
+                kb = inb && has_b && static_cast<double>(sb) >= tau_b;
+            }
             const uint32_t wa = __ballot_sync(0xFFFFFFFFu, ka);
             const uint32_t wb = __ballot_sync(0xFFFFFFFFu, kb);
             if (lane == 0) {
@@ -742,26 +980,46 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 cnt_a += __popc(wa);
                 cnt_b += __popc(wb);
             }
-            if (inb) {
-                if (p.dbg_proxy) {
-                    p.dbg_proxy[unit_a * Nk + j] = sa;
-                    if (has_b) p.dbg_proxy[(unit_a + 1) * Nk + j] = sb;
-                }
-                if (p.dbg_mask) {
-                    p.dbg_mask[unit_a * Nk + j] = ka;
-                    if (has_b) p.dbg_mask[(unit_a + 1) * Nk + j] = kb;
-                }
+            if (inb && p.dbg_proxy) {
+                p.dbg_proxy[unit_a * Nk + j] = sa;
+                if (has_b) p.dbg_proxy[(unit_a + 1) * Nk + j] = sb;
             }
         }
         if (lane == 0) {
             atomicAdd(&m.count_a, cnt_a);
             atomicAdd(&m.count_b, cnt_b);
         }
+        if (by_rank) {
+            min_a = __reduce_min_sync(0xFFFFFFFFu, min_a);
+            min_b = __reduce_min_sync(0xFFFFFFFFu, min_b);
+            if (lane == 0) {
+                atomicMin(&m.sel_min[0], min_a);
+                atomicMin(&m.sel_min[1], min_b);
+            }
+        }
     }
     __syncthreads();
+    if (by_rank) {
+        if (tid == 0) thin_ties(m.mask_a, row_a, Nk, m, 0, &m.count_a);
+        if (tid == 32) thin_ties(m.mask_b, row_b, Nk, m, 1, &m.count_b);
+        __syncthreads();
+        for (int wd = tid; wd < nwords; wd += kThreads) m.mask_u[wd] = m.mask_a[wd] | m.mask_b[wd];
+        if (tid == 0 && p.dbg_stats) {
+            // threshold statistic of a rank rule: the score of the last kept block
+            for (int t = 0; t < (has_b ? 2 : 1); ++t)
+                p.dbg_stats[(unit_a + t) * 3 + 2] =
+                    (t ? m.count_b : m.count_a) == 0 ? INFINITY : key_score(m.sel_min[t]);
+        }
+        __syncthreads();
+    }
+    if (p.dbg_mask) {
+        for (int j = tid; j < Nk; j += kThreads) {
+            p.dbg_mask[unit_a * Nk + j] = (m.mask_a[j >> 5] >> (j & 31)) & 1u;
+            if (has_b) p.dbg_mask[(unit_a + 1) * Nk + j] = (m.mask_b[j >> 5] >> (j & 31)) & 1u;
+        }
+    }
     // correction chunks that still hold a block skipped by tile A (or by an existing tile B)
     {
-        const int nwords = (Nk + 31) >> 5;
         for (int c = tid; c < p.nchunks; c += kThreads) {
             uint32_t need = 0;
             for (int h = 0; h < 2; ++h) {
@@ -841,6 +1099,9 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     p.dbg_stats = L.dbg_stats;
     p.fault_flags = L.fault_flags;
     p.timeout_ns = L.timeout_ns;
+    p.route = L.route;
+    p.topk = L.topk;
+    p.topp = L.topp;
     const long long grid = static_cast<long long>(p.npairs) * L.BH;
     if (grid <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     sol_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(

@@ -87,6 +87,51 @@ sol_status sol_attn_fwd_betas(const void *q, const void *k, const void *v, int B
                               int d, const float *beta_per_head, void *workspace, void *out,
                               int32_t *density_out, void *stream);
 
+/* Block-selection rules.  SOL_ROUTE_THRESHOLD is the paper's rule (keep S_ij >= mu_i + beta*sigma_i).
+ * SOL_ROUTE_TOPK and SOL_ROUTE_TOPP are the two prior-art rules the paper's routing paragraph
+ * contrasts it with (a fixed number of blocks per query; blocks until their cumulative probability
+ * reaches a threshold).  They run on the same proxy row inside the same fused kernel; only the
+ * keep decision differs.  Readings fixed by this library:
+ *   - blocks are ranked by proxy score, highest first; equal scores (-0.0 equals +0.0) rank the
+ *     lower block index first;
+ *   - top-k keeps the first min(k, Nk) blocks of every query tile's row;
+ *   - top-p gives block j the probability w_j / Z, w_j = exp(S_ij - max_j S_ij) in double,
+ *     Z = sum_j w_j (no weighting by token count), and keeps the shortest prefix of the ranking
+ *     whose probability reaches p (block j is kept iff the mass ranked before it is < p*Z);
+ *     p <= 0 keeps none, p >= 1 keeps every block.  The float64 sums are accumulated in an
+ *     unspecified order, so a prefix whose mass lies within about 1e-12*Z of p*Z may end one
+ *     block earlier or later than an exact evaluation;
+ *   - skipped blocks get the same pooled correction term as under the threshold rule. */
+typedef enum {
+    SOL_ROUTE_THRESHOLD = 0,
+    SOL_ROUTE_TOPK = 1,
+    SOL_ROUTE_TOPP = 2
+} sol_route;
+
+/* sol_attn_fwd with the top-k rule: k_blocks >= 0 blocks kept per query tile (values above Nk keep
+ * every block).  density_out then holds min(k_blocks, Nk) for every tile.  Negative k_blocks:
+ * SOL_ERR_INVALID_ARG.  Other arguments as for sol_attn_fwd. */
+sol_status sol_attn_fwd_topk(const void *q, const void *k, const void *v, int B, int H, int N,
+                             int d, int k_blocks, void *workspace, void *out,
+                             int32_t *density_out, void *stream);
+
+/* sol_attn_fwd with the top-p rule: p is the probability mass to cover per query tile (any
+ * non-NaN float; see sol_route for <= 0 and >= 1).  NaN p: SOL_ERR_INVALID_ARG. */
+sol_status sol_attn_fwd_topp(const void *q, const void *k, const void *v, int B, int H, int N,
+                             int d, float p, void *workspace, void *out, int32_t *density_out,
+                             void *stream);
+
+/* sol_attn_fwd_debug for any rule: route selects the rule and param is its parameter (beta for
+ * SOL_ROUTE_THRESHOLD, k for SOL_ROUTE_TOPK -- an integral value >= 0 --, p for SOL_ROUTE_TOPP).
+ * Debug outputs as for sol_attn_fwd_debug; for the rank rules stats_out[...,2] holds the score of
+ * the last kept block (+inf when none is kept) instead of mu + beta*sigma.  Synchronises the
+ * stream and returns the device status.  An unknown route or an invalid param:
+ * SOL_ERR_INVALID_ARG. */
+sol_status sol_attn_fwd_debug_route(const void *q, const void *k, const void *v, int B, int H,
+                                    int N, int d, int route, float param, void *workspace,
+                                    void *out, int32_t *density_out, float *proxy_out,
+                                    uint8_t *mask_out, float *stats_out, void *stream);
+
 /* Test/diagnostic variant of sol_attn_fwd: the same computation plus optional debug outputs,
  * then a stream synchronisation and a read of the device status.  Not for production use.
  *   proxy_out  device float [B,H,Nq,Nk]: the proxy rows S_ij (or NULL)

@@ -137,3 +137,125 @@ def check_parity(q, k, v, beta: float, g: dict, units: np.ndarray, report: dict 
     assert max_abs <= MAX_ABS, max_abs
     assert mean_abs <= MEAN_ABS, mean_abs
     return max_abs, mean_abs, near_total
+
+
+# ------------------------------------------------------------------ top-k / top-p routing rules
+
+TOPP_MASS_BAND = 1e-9     # float64 mass sums in a different order: decisions this close to p*Z may differ
+TOPP_MASS_TOL = 1e-4      # proxy differences (<= 1e-5) move the masses, checked on the oracle's proxy
+
+
+def gpu_run_rule(q, k, v, rule: str, param, units=None):
+    """Pool + forward with a rank rule through the production entry point (sol_attn_fwd_topk /
+    sol_attn_fwd_topp) and the debug entry point; both must agree bit for bit."""
+    B, H, N, d = q.shape
+    Nq = (N + T - 1) // T
+    tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+    ws = torch.zeros(sol.sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+    out = torch.full_like(tq, float("nan"))
+    dens = torch.full((B, H, Nq), -1, dtype=torch.int32, device="cuda")
+    sol.sol_attn_pool(tk, tv, ws)
+    if rule == "topk":
+        sol.sol_attn_fwd_topk(tq, tk, tv, int(param), ws, out, dens)
+    else:
+        sol.sol_attn_fwd_topp(tq, tk, tv, float(param), ws, out, dens)
+    st, where = sol.sol_attn_read_status(ws)
+    assert st == 0, (sol.STATUS.get(st), where)
+    out2 = torch.full_like(tq, float("nan"))
+    dens2 = torch.full((B, H, Nq), -1, dtype=torch.int32, device="cuda")
+    proxy = torch.full((B, H, Nq, Nq), float("nan"), dtype=torch.float32, device="cuda")
+    mask = torch.full((B, H, Nq, Nq), 255, dtype=torch.uint8, device="cuda")
+    stats = torch.full((B, H, Nq, 3), float("nan"), dtype=torch.float32, device="cuda")
+    st = sol.sol_attn_fwd_debug_route(tq, tk, tv, rule, float(param), ws, out2, dens2, proxy, mask, stats)
+    assert st == 0, sol.STATUS.get(st)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16)), "debug/production outputs differ"
+    assert torch.equal(dens, dens2)
+    if units is None:
+        units = np.arange(B * H * Nq, dtype=np.int64)
+    sel = torch.as_tensor(np.asarray(units), device="cuda")
+    pick = lambda t: t.reshape(B * H * Nq, *t.shape[3:]).index_select(0, sel).cpu().numpy()
+    pad = Nq * T - N
+    o = torch.nn.functional.pad(out.view(B * H, N, d), (0, 0, 0, pad), value=float("nan"))
+    res = dict(units=units, density=dens.cpu().numpy(), mask=pick(mask), proxy=pick(proxy),
+               stats=pick(stats),
+               out_units=o.view(B * H * Nq, T, d).index_select(0, sel).float().cpu().numpy())
+    return res
+
+
+def check_rule_parity(q, k, v, rule: str, param, g: dict, report: dict | None = None):
+    """Acceptance for a rank rule, per query tile:
+      - the GPU proxy row matches the oracle's (as for the threshold rule), mu/sigma too;
+      - the GPU mask is exactly the oracle's selection applied to the GPU's own proxy row (top-p:
+        a prefix one block longer or shorter is accepted when the mass sum lies within
+        TOPP_MASS_BAND of p);
+      - against the oracle's own proxy: top-k keeps min(k, Nk) blocks and any disagreement with
+        the oracle's mask lies within BAND of the oracle's k-th score; top-p's kept mass reaches
+        p and drops below it without the lowest kept block, within TOPP_MASS_TOL;
+      - the threshold statistic is the lowest kept GPU score (+inf if none), density = mask sums;
+      - outputs match the oracle's attention under the GPU's mask (MAX_ABS / MEAN_ABS)."""
+    from oracle import sol_ref_routes as rr
+    B, H, N, d = q.shape
+    Nk = (N + T - 1) // T
+    units = g["units"]
+    kbar, vbar = sol_ref.pool(k), sol_ref.pool(v)
+    r = rr.route_variant(q, kbar, rule, param, units)
+    gm = g["mask"].reshape(-1, Nk)
+    gp = g["proxy"].reshape(-1, Nk)
+    gs = g["stats"].reshape(-1, 3)
+    assert np.all((gm == 0) | (gm == 1))
+    np.testing.assert_allclose(gp, r["proxy"], rtol=1e-6, atol=STAT_ATOL)
+    np.testing.assert_allclose(gs[:, 0], r["mu"], rtol=0, atol=STAT_ATOL)
+    np.testing.assert_allclose(gs[:, 1], r["sigma"], rtol=0, atol=STAT_ATOL)
+    cnt = gm.sum(1)
+    assert np.array_equal(g["density"].reshape(-1)[units], cnt.astype(np.int32))
+    low = np.array([gp[u][gm[u] == 1].min() if cnt[u] else np.inf for u in range(len(units))],
+                   np.float32)
+    assert np.array_equal(gs[:, 2], low)
+    band_rows = 0
+    if rule == "topk":
+        want = rr.select_topk(gp, int(param))
+        assert np.array_equal(gm, want), f"{int((gm != want).sum())} blocks differ on the GPU proxy"
+        assert np.all(cnt == min(int(param), Nk))
+        om = r["mask"]
+        for u in np.nonzero((gm != om).any(1))[0]:
+            kk = min(int(param), Nk)
+            kth = np.sort(r["proxy"][u].astype(np.float64))[::-1][kk - 1]
+            diff = np.nonzero(gm[u] != om[u])[0]
+            assert np.all(np.abs(r["proxy"][u, diff] - kth) <= 2 * BAND), (u, diff)
+            band_rows += 1
+    else:
+        p = float(param)
+        want, bound = rr.select_topp(gp, p, with_boundary=True)
+        for u in range(len(units)):
+            if np.array_equal(gm[u], want[u]):
+                continue
+            # the GPU's prefix may end one block away only for a decision at the band
+            lo_b, hi_b = bound[u]
+            near = abs(lo_b - p) <= TOPP_MASS_BAND or abs(hi_b - p) <= TOPP_MASS_BAND
+            assert near and abs(int(gm[u].sum()) - int(want[u].sum())) == 1, u
+            band_rows += 1
+        if 0.0 < p < 1.0:
+            for u in range(len(units)):
+                s = r["proxy"][u].astype(np.float64)
+                w = np.exp(s - s.max())
+                kept = gm[u] == 1
+                frac = w[kept].sum() / w.sum()
+                assert frac >= p - TOPP_MASS_TOL, (u, frac)
+                lowest = np.argmin(np.where(kept, gp[u], np.inf))
+                assert (w[kept].sum() - w[lowest]) / w.sum() < p + TOPP_MASS_TOL, u
+    o = sol_ref.attend(q, k, v, kbar, vbar, units, gm)
+    errs = []
+    for u_i, u in enumerate(units):
+        bh, i = divmod(int(u), Nk)
+        lo, hi = i * T, min(N, (i + 1) * T)
+        got = g["out_units"][u_i, :hi - lo]
+        assert np.all(np.isfinite(got))
+        errs.append(np.abs(got.astype(np.float64) - o[u_i, :hi - lo]))
+    err = np.concatenate(errs)
+    max_abs, mean_abs = float(err.max()), float(err.mean())
+    if report is not None:
+        report.update(max_abs=max_abs, mean_abs=mean_abs, band_rows=band_rows,
+                      density=float(gm.mean()), tile_density_std=float(gm.mean(1).std()))
+    assert max_abs <= MAX_ABS, max_abs
+    assert mean_abs <= MEAN_ABS, mean_abs
+    return max_abs, mean_abs

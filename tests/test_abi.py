@@ -91,3 +91,20 @@ def test_host_entry_rejects_bad_arguments_on_host(lib):
     assert f(A, A, A, 1, 1, 128, 128, C.c_float(0.5), A, A, A, A, A, A, A, None, None) == 1
     assert f(A, A, A, 1, 1, 128, 128, C.c_float(math.nan), A, A, A, A, A, None, A, None, None) == 1
     assert f(A, A, A, 1, 1, 128, 128, C.c_float(0.5), MIS, A, A, A, A, None, A, None, None) == 3
+
+
+def test_rank_rules_reject_bad_parameters_before_launch(lib):
+    """Negative or fractional k, NaN p and unknown rules fail on the host (no GPU needed)."""
+    f = lib.sol_attn_fwd_topk
+    assert f(A, A, A, 1, 1, 128, 128, -1, A, A, None, None) == 1
+    assert f(A, A, A, 1, 1, 128, 96, 3, A, A, None, None) == 2
+    g = lib.sol_attn_fwd_topp
+    assert g(A, A, A, 1, 1, 128, 128, C.c_float(math.nan), A, A, None, None) == 1
+    assert g(None, A, A, 1, 1, 128, 128, C.c_float(0.5), A, A, None, None) == 1
+    h = lib.sol_attn_fwd_debug_route
+    assert h(A, A, A, 1, 1, 128, 128, 3, C.c_float(1.0), A, A, None, None, None, None, None) == 1
+    assert h(A, A, A, 1, 1, 128, 128, 1, C.c_float(2.5), A, A, None, None, None, None, None) == 1
+    assert h(A, A, A, 1, 1, 128, 128, 1, C.c_float(-1.0), A, A, None, None, None, None, None) == 1
+    assert h(A, A, A, 1, 1, 128, 128, 2, C.c_float(math.nan), A, A, None, None, None, None, None) == 1
+    assert h(A, A, A, 1, 1, 128, 128, 0, C.c_float(math.nan), A, A, None, None, None, None, None) == 1
+    assert h(A, A, A, 1, 1, 128, 128, 2, C.c_float(0.5), A, A, None, MIS, None, None, None) == 3
