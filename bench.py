@@ -169,6 +169,72 @@ def flop_counts(mask: np.ndarray, N: int, d: int = 128):
                 density_tokens=density_tokens)
 
 
+def density_spread(dens: np.ndarray, Nk: int) -> dict:
+    """Density statistics of one call from the per-tile kept-block counts [B, H, Nq]: the overall
+    block fraction, its spread over query tiles, and its spread over heads (the page contrasts a
+    stable overall density with top-p's fluctuating one)."""
+    per_tile = dens.reshape(-1, dens.shape[-1]).astype(np.float64) / Nk
+    return {"density": float(per_tile.mean()), "tile_density_std": float(per_tile.std()),
+            "head_density_std": float(per_tile.mean(1).std())}
+
+
+def compare_routes(sol, tq, tk, tv, ws, out, dens, flush, stream, beta: float, steps: int):
+    """Routing rules at one matched overall density: the threshold rule at ``beta`` sets it;
+    per-head betas (calibrated), top-k (k = density * Nk) and top-p (p found by bisection) are
+    brought to the same density; each is timed (fwd only, L2 flushed) and its spread reported."""
+    import torch
+    from free_sparse_attention_block_b200 import calibrate
+
+    B, H, N, d = tq.shape
+    Nk = dens.shape[-1]
+    runs = {
+        "threshold": lambda: sol.sol_attn_fwd(tq, tk, tv, beta, ws, out, dens),
+    }
+
+    def measure(fn):
+        fn()
+        torch.cuda.synchronize()
+        return dens.cpu().numpy()
+
+    target = density_spread(measure(runs["threshold"]), Nk)["density"]
+    t0 = time.perf_counter()
+    betas, _ = calibrate.calibrate_betas(tq, tk, tv, target)
+    calib_s = time.perf_counter() - t0
+    runs["per_head_beta"] = lambda: sol.sol_attn_fwd_betas(tq, tk, tv, betas, ws, out, dens)
+    k_match = max(1, int(round(target * Nk)))
+    runs["topk"] = lambda: sol.sol_attn_fwd_topk(tq, tk, tv, k_match, ws, out, dens)
+    lo, hi = 0.0, 1.0
+    for _ in range(30):
+        mid = 0.5 * (lo + hi)
+        got = density_spread(measure(lambda: sol.sol_attn_fwd_topp(tq, tk, tv, mid, ws, out, dens)), Nk)
+        if got["density"] < target:
+            lo = mid
+        else:
+            hi = mid
+    p_match = hi
+    runs["topp"] = lambda: sol.sol_attn_fwd_topp(tq, tk, tv, p_match, ws, out, dens)
+    params = {"threshold": beta, "per_head_beta": "calibrated", "topk": k_match, "topp": p_match}
+    res = []
+    for name, fn in runs.items():
+        stats = density_spread(measure(fn), Nk)
+        ts = []
+        for _ in range(max(3, steps)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in ts]))
+        res.append({"rule": name, "param": params[name], "fwd_ms": round(ms, 4)} |
+                   {k2: round(v2, 5) for k2, v2 in stats.items()})
+    st, where = sol.sol_attn_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {sol.STATUS.get(st)} at wait site {where}")
+    return {"target_density": round(target, 5), "calibration_s": round(calib_s, 3), "rules": res}
+
+
 # ------------------------------------------------------------------------------ oracle arm
 
 def oracle_sample(wl, beta: float, q, k, v, ntiles: int, seed: int = 0):
@@ -378,6 +444,12 @@ def run_ours(args, wl):
                           "dense_equiv_tflops": round(dense / (ms * 1e-3) / 1e12, 1),
                           "computed_tile_frac": round(fc2["kept"] / (ms * 1e-3) / 1e12 / PEAK_BF16, 4)})
 
+    # ---- routing rules at matched density (threshold, per-head beta, top-k, top-p), for the record
+    routes = None
+    if not args.no_route_compare:
+        routes = compare_routes(sol, tq, tk, tv, ws, out, dens, flush, stream, args.beta,
+                                max(3, args.steps // 2))
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -424,6 +496,8 @@ def run_ours(args, wl):
     }
     if sweep:
         line["sweep"] = sweep
+    if routes:
+        line["routing_compare"] = routes
     print(json.dumps(line), flush=True)
 
 
@@ -444,6 +518,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU-baseline sample time")
     ap.add_argument("--ref-seconds", type=float, default=90.0, help="target total time of the oracle arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-route-compare", action="store_true",
+                    help="skip the routing-rule comparison at matched density")
     ap.add_argument("--head-dim", type=int, choices=[64, 128], default=None,
                     help="generate the workload with this head dimension instead of its own")
     args = ap.parse_args()

@@ -724,7 +724,9 @@ __device__ __forceinline__ void load_vec(const float *src, float (&x)[LC])
     }
 }
 
-template <int D>
+// kRank: the top-k / top-p rules (radix selection) are compiled in; the threshold rule's kernel is
+// a separate instantiation without that code, which otherwise costs it about 3 % (measured).
+template <int D, bool kRank>
 __global__ void __launch_bounds__(kThreads, 2)
 sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
@@ -948,8 +950,8 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncthreads();
     // ---------------- routing 4: keep masks (ballot per 32 blocks), counts, debug rows
-    const bool by_rank = p.route != kRouteThreshold;   // top-k / top-p instead of mu + beta*sigma
-    if (by_rank) radix_select(row_a, row_b, has_b, Nk, m, p);
+    constexpr bool by_rank = kRank;   // top-k / top-p instead of mu + beta*sigma
+    if constexpr (by_rank) radix_select(row_a, row_b, has_b, Nk, m, p);
     const int nwords = (Nk + 31) >> 5;
     {
         const double tau_a = m.tau[0], tau_b = m.tau[1];
@@ -961,7 +963,7 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float sa = inb ? row_a[j] : 0.0f;
             const float sb = inb ? row_b[j] : 0.0f;
             bool ka, kb;
-            if (by_rank) {
+            if constexpr (by_rank) {
                 const uint32_t ya = score_key(sa), yb = score_key(sb);
                 ka = inb && sel_keep(m, 0, ya);
                 kb = inb && has_b && sel_keep(m, 1, yb);
@@ -989,7 +991,7 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             atomicAdd(&m.count_a, cnt_a);
             atomicAdd(&m.count_b, cnt_b);
         }
-        if (by_rank) {
+        if constexpr (by_rank) {
             min_a = __reduce_min_sync(0xFFFFFFFFu, min_a);
             min_b = __reduce_min_sync(0xFFFFFFFFu, min_b);
             if (lane == 0) {
@@ -999,7 +1001,7 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     }
     __syncthreads();
-    if (by_rank) {
+    if constexpr (by_rank) {
         if (tid == 0) thin_ties(m.mask_a, row_a, Nk, m, 0, &m.count_a);
         if (tid == 32) thin_ties(m.mask_b, row_b, Nk, m, 1, &m.count_b);
         __syncthreads();
@@ -1061,7 +1063,7 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int D>
+template <int D, bool kRank>
 cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
 {
     static std::once_flag attr_once[64];
@@ -1072,7 +1074,7 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     constexpr uint32_t kSmem = smem_bytes<D>();
     cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once[dev], [&] {
-        attr_err = cudaFuncSetAttribute(sol_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(sol_fwd_kernel<D, kRank>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(kSmem));
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -1104,7 +1106,7 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     p.topp = L.topp;
     const long long grid = static_cast<long long>(p.npairs) * L.BH;
     if (grid <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    sol_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(
+    sol_fwd_kernel<D, kRank><<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(
         *L.tm_q, *L.tm_k, *L.tm_v, *L.tm_kb, *L.tm_vb, p);
     return cudaGetLastError();
 }
@@ -1113,8 +1115,9 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
 
 cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream)
 {
-    if (L.d == 128) return launch_d<128>(L, stream);
-    if (L.d == 64) return launch_d<64>(L, stream);
+    const bool rank = L.route != kRouteThreshold;
+    if (L.d == 128) return rank ? launch_d<128, true>(L, stream) : launch_d<128, false>(L, stream);
+    if (L.d == 64) return rank ? launch_d<64, true>(L, stream) : launch_d<64, false>(L, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -58,3 +58,13 @@ def test_max_over_ranks_gloo_two_ranks():
     mp.start_processes(_worker, args=(2, port, times, out), nprocs=2, start_method="spawn", join=True)
     assert out[0] == out[1] == 3.5
     assert bench.max_over_ranks(2.0) == 2.0        # no process group: unchanged
+
+
+def test_density_spread_hand_computed():
+    # 2 heads x 3 tiles over Nk = 4 blocks: head 0 keeps 1,2,3 blocks, head 1 keeps 2,2,2
+    dens = np.array([[[1, 2, 3], [2, 2, 2]]], np.int32)
+    s = bench.density_spread(dens, 4)
+    tiles = np.array([1, 2, 3, 2, 2, 2]) / 4
+    assert abs(s["density"] - 0.5) < 1e-15
+    assert abs(s["tile_density_std"] - tiles.std()) < 1e-15
+    assert s["head_density_std"] == 0.0          # both heads average 0.5
