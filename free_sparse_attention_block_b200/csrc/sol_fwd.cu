@@ -8,9 +8,10 @@
 // sparse attention, and skipped blocks are approximated rather than dropped).
 //
 // One CTA owns one 128-row MMA tile = two adjacent 64-row routing tiles (A: rows 0-63, B: rows
-// 64-127) of one head.  Two CTAs fit on an SM (at most about 104 KB of shared memory and 256 TMEM
-// columns each), so one CTA's routing and softmax overlap the other's tensor-core work.  The
-// kernel is compiled for head dimensions d = 128 and d = 64 (template parameter D).
+// 64-127) of one head.  Two CTAs fit on an SM (about 110 KB of shared memory at d = 128, 94 KB at
+// d = 64, and 256 TMEM columns each), so one CTA's routing and softmax overlap the other's
+// tensor-core work.  The kernel is compiled for head dimensions d = 128 and d = 64 (template
+// parameter D), and for the threshold rule or the top-k / top-p rules (template parameter kRank).
 //
 //  1. Routing (all 6 warps).  TMA brings the Q tile into shared memory; q_bar of each routing
 //     tile is summed from it in float32; every warp computes proxy scores
