@@ -256,7 +256,9 @@ def oracle_sample(wl, beta: float, q, k, v, ntiles: int, seed: int = 0):
     rng = np.random.default_rng(seed)
     BH = wl.B * wl.H
     Nq = wl.nq
-    heads = sorted(set(int(h) for h in rng.integers(0, BH, size=max(1, min(BH, ntiles // 8)))))
+    # distinct heads, enough of them to hold ntiles tiles (and at least ntiles // 8 of them)
+    nh = min(BH, max(1, ntiles // 8, -(-ntiles // Nq)))
+    heads = sorted(int(h) for h in rng.choice(BH, size=nh, replace=False))
     per = int(math.ceil(ntiles / len(heads)))
     qh = q.reshape(BH, wl.N, wl.d)
     kh = k.reshape(BH, wl.N, wl.d)
@@ -527,9 +529,7 @@ def main():
     ap.add_argument("--workload", default="mid", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--beta", type=float, default=0.5)
     ap.add_argument("--sweep", action="store_true", help="also time fwd over the workload's beta sweep")
-    ap.add_argument("--cpu-seconds", type=float, default=20.0,
-                    help="target CPU-baseline sample time (the estimate from a short probe runs long; "
-                         "about 10 s of oracle work results)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline sample time")
     ap.add_argument("--ref-seconds", type=float, default=90.0, help="target total time of the oracle arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-route-compare", action="store_true",
