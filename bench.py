@@ -256,8 +256,9 @@ def oracle_sample(wl, beta: float, q, k, v, ntiles: int, seed: int = 0):
     rng = np.random.default_rng(seed)
     BH = wl.B * wl.H
     Nq = wl.nq
-    # distinct heads, enough of them to hold ntiles tiles (and at least ntiles // 8 of them)
-    nh = min(BH, max(1, ntiles // 8, -(-ntiles // Nq)))
+    # whole heads where possible (each sampled head's K and V are pooled once, as in the full
+    # job), distinct, as many as ntiles needs
+    nh = min(BH, max(1, -(-ntiles // Nq)))
     heads = sorted(int(h) for h in rng.choice(BH, size=nh, replace=False))
     per = int(math.ceil(ntiles / len(heads)))
     qh = q.reshape(BH, wl.N, wl.d)
