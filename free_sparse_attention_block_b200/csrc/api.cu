@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -99,28 +100,45 @@ struct RouteArg {
     float topp = 0.0f;
 };
 
-sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
-                   float beta, const float *beta_head, void *workspace, void *out, int32_t *density,
-                   float *dbg_proxy, uint8_t *dbg_mask, float *dbg_stats, int fault_flags,
-                   unsigned long long timeout_ns, cudaStream_t stream, RouteArg ra = RouteArg{})
-{
-    Shape s{};
-    sol_status st = check_shape(B, H, N, d, &s);
-    if (st != SOL_OK) return st;
-    if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
-    st = check_ptrs({q, k, v, workspace, out});
-    if (st != SOL_OK) return st;
-    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
-    if (density && (reinterpret_cast<uintptr_t>(density) & 3u)) return SOL_ERR_ALIGNMENT;
-    if (beta_head && (reinterpret_cast<uintptr_t>(beta_head) & 3u)) return SOL_ERR_ALIGNMENT;
+// Device pointers of the pooled arrays and status words for heads [bh0, bh0 + count) of a call
+// whose workspace is laid out for the shape `full`.
+struct Pooled {
+    float *k32, *v32;
+    uint8_t *k16, *v16;
+    DeviceStatus *status;
+};
 
-    const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk, s.d);
+Pooled pooled_at(void *workspace, const Shape &full, int bh0)
+{
+    const WorkspaceLayout wl = workspace_layout(full.BH, full.Nk, full.d);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t off = static_cast<size_t>(bh0) * static_cast<size_t>(full.Nk) * static_cast<size_t>(full.d);
+    Pooled p{};
+    p.k32 = reinterpret_cast<float *>(ws + wl.kbar32) + off;
+    p.v32 = reinterpret_cast<float *>(ws + wl.vbar32) + off;
+    p.k16 = ws + wl.kbar16 + off * 2;
+    p.v16 = ws + wl.vbar16 + off * 2;
+    p.status = reinterpret_cast<DeviceStatus *>(ws);
+    return p;
+}
+
+// Pool K, V of the s.BH heads starting at k, v into `pw` (no argument checks).
+sol_status launch_pool(const void *k, const void *v, const Shape &s, const Pooled &pw, cudaStream_t stream)
+{
+    return launch_pool_kv(k, v, s.BH, s.N, s.Nk, s.d, pw.k32, pw.v32, pw.k16, pw.v16, stream) == cudaSuccess
+               ? SOL_OK : SOL_ERR_CUDA;
+}
+
+// Fused forward over the s.BH heads starting at q, k, v, out, density (no argument checks).
+sol_status launch_fwd(const void *q, const void *k, const void *v, const Shape &s, const Pooled &pw,
+                      float beta, const float *beta_head, void *out, int32_t *density,
+                      float *dbg_proxy, uint8_t *dbg_mask, float *dbg_stats, int fault_flags,
+                      unsigned long long timeout_ns, cudaStream_t stream, const RouteArg &ra)
+{
     CUtensorMap tq, tk, tv, tkb, tvb;
     if (!encode_rows(&tq, q, s.N, s.BH, 128, s.d) || !encode_rows(&tk, k, s.N, s.BH, kTile, s.d) ||
-        !encode_rows(&tv, v, s.N, s.BH, kTile, s.d) ||
-        !encode_rows(&tkb, ws + wl.kbar16, s.Nk, s.BH, kTile, s.d) ||
-        !encode_rows(&tvb, ws + wl.vbar16, s.Nk, s.BH, kTile, s.d))
+        !encode_rows(&tv, v, s.N, s.BH, kTile, s.d) || !encode_rows(&tkb, pw.k16, s.Nk, s.BH, kTile, s.d) ||
+        !encode_rows(&tvb, pw.v16, s.Nk, s.BH, kTile, s.d))
         return SOL_ERR_CUDA;
     FwdLaunch L{};
     L.tm_q = &tq;
@@ -135,10 +153,10 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     L.d = s.d;
     L.beta = beta;
     L.beta_head = beta_head;
-    L.kbar32 = reinterpret_cast<const float *>(ws + wl.kbar32);
+    L.kbar32 = pw.k32;
     L.out = out;
     L.density = density;
-    L.status = reinterpret_cast<DeviceStatus *>(ws);
+    L.status = pw.status;
     L.dbg_proxy = dbg_proxy;
     L.dbg_mask = dbg_mask;
     L.dbg_stats = dbg_stats;
@@ -148,6 +166,24 @@ sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, in
     L.topk = ra.topk;
     L.topp = ra.topp;
     return launch_sol_fwd(L, stream) == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
+
+sol_status run_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                   float beta, const float *beta_head, void *workspace, void *out, int32_t *density,
+                   float *dbg_proxy, uint8_t *dbg_mask, float *dbg_stats, int fault_flags,
+                   unsigned long long timeout_ns, cudaStream_t stream, RouteArg ra = RouteArg{})
+{
+    Shape s{};
+    sol_status st = check_shape(B, H, N, d, &s);
+    if (st != SOL_OK) return st;
+    if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
+    st = check_ptrs({q, k, v, workspace, out});
+    if (st != SOL_OK) return st;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
+    if (density && (reinterpret_cast<uintptr_t>(density) & 3u)) return SOL_ERR_ALIGNMENT;
+    if (beta_head && (reinterpret_cast<uintptr_t>(beta_head) & 3u)) return SOL_ERR_ALIGNMENT;
+    return launch_fwd(q, k, v, s, pooled_at(workspace, s, 0), beta, beta_head, out, density, dbg_proxy,
+                      dbg_mask, dbg_stats, fault_flags, timeout_ns, stream, ra);
 }
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000ull * 1000ull * 1000ull;   // 2 s
@@ -170,6 +206,43 @@ sol_status route_arg(int route, double param, RouteArg *ra)
         return SOL_OK;
     }
     return SOL_ERR_INVALID_ARG;
+}
+
+// Copy streams and events of the pipelined host entry point: one set per device, created on first
+// use and kept until the process exits.
+constexpr int kHostGroups = 8;
+
+struct HostPipe {
+    std::once_flag once;
+    std::mutex mu;          // one enqueue at a time per device (the events are reused)
+    cudaError_t err = cudaSuccess;
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t uploaded[kHostGroups] = {};
+    cudaEvent_t computed[kHostGroups] = {};
+};
+
+HostPipe g_host_pipes[64];
+
+HostPipe *host_pipe()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    HostPipe &hp = g_host_pipes[dev];
+    std::call_once(hp.once, [&hp] {
+        auto event = [&hp](cudaEvent_t *e) {
+            if (hp.err == cudaSuccess) hp.err = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+        };
+        hp.err = cudaStreamCreateWithFlags(&hp.up, cudaStreamNonBlocking);
+        if (hp.err == cudaSuccess) hp.err = cudaStreamCreateWithFlags(&hp.down, cudaStreamNonBlocking);
+        event(&hp.start);
+        event(&hp.done);
+        for (int g = 0; g < kHostGroups; ++g) {
+            event(&hp.uploaded[g]);
+            event(&hp.computed[g]);
+        }
+    });
+    return hp.err == cudaSuccess ? &hp : nullptr;
 }
 
 }  // namespace
@@ -196,13 +269,8 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
     if (st != SOL_OK) return st;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    const WorkspaceLayout wl = workspace_layout(s.BH, s.Nk, s.d);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    if (cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), cs) != cudaSuccess) return SOL_ERR_CUDA;
-    cudaError_t e = launch_pool_kv(k, v, s.BH, s.N, s.Nk, s.d, reinterpret_cast<float *>(ws + wl.kbar32),
-                                   reinterpret_cast<float *>(ws + wl.vbar32), ws + wl.kbar16,
-                                   ws + wl.vbar16, cs);
-    return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), cs) != cudaSuccess) return SOL_ERR_CUDA;
+    return launch_pool(k, v, s, pooled_at(workspace, s, 0), cs);
 }
 
 sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
@@ -302,21 +370,58 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
         return SOL_ERR_INVALID_ARG;
     st = check_ptrs({d_q, d_k, d_v, workspace, d_out});
     if (st != SOL_OK) return st;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
+    if (d_density && (reinterpret_cast<uintptr_t>(d_density) & 3u)) return SOL_ERR_ALIGNMENT;
     if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    const size_t bytes = static_cast<size_t>(s.BH) * s.N * s.d * 2;
-    if (cudaMemcpyAsync(d_q, h_q, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-        cudaMemcpyAsync(d_k, h_k, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-        cudaMemcpyAsync(d_v, h_v, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    HostPipe *hp = host_pipe();
+    if (!hp) return SOL_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(hp->mu);
+
+    // Heads are split into up to kHostGroups contiguous groups.  Group g's inputs are uploaded on
+    // the `up` stream; `stream` pools and runs the forward for g once they have landed (while the
+    // next groups upload); its output is downloaded on the `down` stream while later groups
+    // compute.  The last download is joined back into `stream`.
+    const int G = std::min(s.BH, kHostGroups);
+    const size_t head_bytes = static_cast<size_t>(s.N) * static_cast<size_t>(s.d) * 2;
+    const size_t head_dens = static_cast<size_t>(s.Nq) * sizeof(int32_t);
+    auto fail = [](cudaError_t e) { return e != cudaSuccess; };
+    if (fail(cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), cs)) ||
+        fail(cudaEventRecord(hp->start, cs)) || fail(cudaStreamWaitEvent(hp->up, hp->start, 0)) ||
+        fail(cudaStreamWaitEvent(hp->down, hp->start, 0)))
         return SOL_ERR_CUDA;
-    st = sol_attn_pool(d_k, d_v, B, H, N, d, workspace, stream);
-    if (st != SOL_OK) return st;
-    st = sol_attn_fwd(d_q, d_k, d_v, B, H, N, d, beta, workspace, d_out, d_density, stream);
-    if (st != SOL_OK) return st;
-    if (cudaMemcpyAsync(h_out, d_out, bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return SOL_ERR_CUDA;
-    if (h_density &&
-        cudaMemcpyAsync(h_density, d_density, static_cast<size_t>(s.BH) * s.Nq * sizeof(int32_t),
-                        cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    for (int g = 0; g < G; ++g) {
+        const int h0 = static_cast<int>(static_cast<long long>(s.BH) * g / G);
+        const int h1 = static_cast<int>(static_cast<long long>(s.BH) * (g + 1) / G);
+        const size_t off = static_cast<size_t>(h0) * head_bytes;
+        const size_t bytes = static_cast<size_t>(h1 - h0) * head_bytes;
+        uint8_t *gq = static_cast<uint8_t *>(d_q) + off;
+        uint8_t *gk = static_cast<uint8_t *>(d_k) + off;
+        uint8_t *gv = static_cast<uint8_t *>(d_v) + off;
+        uint8_t *go = static_cast<uint8_t *>(d_out) + off;
+        if (fail(cudaMemcpyAsync(gq, static_cast<const uint8_t *>(h_q) + off, bytes, cudaMemcpyHostToDevice, hp->up)) ||
+            fail(cudaMemcpyAsync(gk, static_cast<const uint8_t *>(h_k) + off, bytes, cudaMemcpyHostToDevice, hp->up)) ||
+            fail(cudaMemcpyAsync(gv, static_cast<const uint8_t *>(h_v) + off, bytes, cudaMemcpyHostToDevice, hp->up)) ||
+            fail(cudaEventRecord(hp->uploaded[g], hp->up)) || fail(cudaStreamWaitEvent(cs, hp->uploaded[g], 0)))
+            return SOL_ERR_CUDA;
+        Shape gs = s;
+        gs.BH = h1 - h0;
+        const Pooled pw = pooled_at(workspace, s, h0);
+        int32_t *gd = d_density ? d_density + static_cast<size_t>(h0) * s.Nq : nullptr;
+        st = launch_pool(gk, gv, gs, pw, cs);
+        if (st == SOL_OK)
+            st = launch_fwd(gq, gk, gv, gs, pw, beta, nullptr, go, gd, nullptr, nullptr, nullptr, 0,
+                            kDefaultTimeoutNs, cs, RouteArg{});
+        if (st != SOL_OK) return st;
+        if (fail(cudaEventRecord(hp->computed[g], cs)) || fail(cudaStreamWaitEvent(hp->down, hp->computed[g], 0)) ||
+            fail(cudaMemcpyAsync(static_cast<uint8_t *>(h_out) + off, go, bytes, cudaMemcpyDeviceToHost, hp->down)))
+            return SOL_ERR_CUDA;
+        if (h_density &&
+            fail(cudaMemcpyAsync(h_density + static_cast<size_t>(h0) * s.Nq, gd,
+                                 static_cast<size_t>(h1 - h0) * head_dens, cudaMemcpyDeviceToHost, hp->down)))
+            return SOL_ERR_CUDA;
+    }
+    if (fail(cudaEventRecord(hp->done, hp->down)) || fail(cudaStreamWaitEvent(cs, hp->done, 0)))
         return SOL_ERR_CUDA;
     return SOL_OK;
 }

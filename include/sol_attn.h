@@ -31,8 +31,9 @@
  *     launch.  SOL_ERR_CUDA means a CUDA runtime/driver call or launch failed.
  *   - Device-side failures (a pipeline wait that ran out of time) are recorded in a status word
  *     inside the workspace; sol_attn_read_status() synchronises the stream and returns it.
- *   - The library keeps no state between calls apart from per-device one-time set-up
- *     (kernel attributes, the driver entry point for tensor-map encoding); it is thread-safe.
+ *   - The library keeps no state between calls apart from per-device one-time set-up (kernel
+ *     attributes, the driver entry point for tensor-map encoding, and the two copy streams and
+ *     the events sol_attn_fwd_host pipelines its copies with); it is thread-safe.
  */
 #ifndef SOL_ATTN_H
 #define SOL_ATTN_H
@@ -152,9 +153,15 @@ sol_status sol_attn_fwd_debug(const void *q, const void *k, const void *v, int B
 sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream);
 
 /* One end-to-end call on host buffers: copies q, k, v from (preferably pinned) host memory into
- * the caller's device buffers, pools, runs the forward, and copies out and density back, all
- * queued on `stream` without synchronising.  Host buffers must stay valid until the stream
- * reaches this point.  h_density / d_density may both be NULL. */
+ * the caller's device buffers, pools, runs the forward, and copies out and density back, without
+ * synchronising.  The heads are split into up to 8 contiguous groups and the copies are pipelined
+ * with the compute: group g+1 uploads on an internal copy stream while `stream` pools and runs
+ * group g, and group g's output downloads on a second internal copy stream while later groups
+ * compute.  The uploads wait for all work queued on `stream` before this call, and everything
+ * (the last download included) is ordered before work queued on `stream` after it, so the device
+ * buffers may be reused by the next call.  Host buffers must stay valid until `stream` reaches
+ * that point.  h_density / d_density may both be NULL.  workspace: 256-byte aligned, as for
+ * sol_attn_pool.  Results are bit-identical to sol_attn_pool + sol_attn_fwd. */
 sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, int B, int H,
                              int N, int d, float beta, void *d_q, void *d_k, void *d_v,
                              void *workspace, void *d_out, int32_t *d_density, void *h_out,
