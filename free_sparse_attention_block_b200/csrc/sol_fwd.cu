@@ -58,8 +58,8 @@ constexpr uint32_t kKVHalfBytes = kTile * 64 * 2;      // 64 rows x 64 channels,
 constexpr int kStages = 2;
 
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemO = 128;                       // O accumulator: columns 128..128+d-1
-__device__ __forceinline__ uint32_t tmem_s_col(int b) { return b ? 64u : 0u; }
+constexpr int kMaxSBufs = 3;
+__device__ __forceinline__ uint32_t tmem_s_col(int b) { return 64u * static_cast<uint32_t>(b); }
 
 constexpr float kRescaleLog2 = 8.0f;                   // rescale O only if the max grows > 2^8
 
@@ -94,9 +94,14 @@ struct Geo {
     static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, 64, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
     static constexpr int kOChunks = D / 32;              // 32-column TMEM loads of a row of O
+    // S buffers of 64 columns in TMEM, then O (D columns): three buffers fit next to a 64-column O
+    // (the MMA warp then issues QK two items ahead), two next to a 128-column one
+    static constexpr int kSBufs = D == 64 ? 3 : 2;
+    static constexpr uint32_t kTmemO = 64u * kSBufs;
     static constexpr int kLaneCh = D / 32;               // channels per lane in the proxy dot products
     static_assert(kOffMisc % 1024 == 0, "shared-memory tiles need 1024-byte alignment");
-    static_assert(kTmemO + D <= kTmemCols, "O accumulator must fit in the TMEM allocation");
+    static_assert(kTmemO + D <= kTmemCols, "S buffers and O must fit in the TMEM allocation");
+    static_assert(kSBufs <= kMaxSBufs, "barrier arrays");
 };
 
 enum SelState : int { kSelRun = 0, kSelNone = 1, kSelAll = 2 };
@@ -111,7 +116,7 @@ struct Misc {
     double red[2][kNumWarps];
     double mu[2], sigma[2], tau[2];
     uint64_t q_full, k_full[kStages], v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2], o_final, drain, never;
+    uint64_t s_full[kMaxSBufs], p_full[kMaxSBufs], o_final, drain, never;
     uint32_t mask_a[kMaskWords];
     uint32_t mask_b[kMaskWords];
     uint32_t mask_u[kMaskWords];
@@ -181,39 +186,34 @@ __device__ bool wait_bar(uint64_t *bar, uint32_t parity, Misc &m, const Params &
     }
 }
 
-// Smallest set bit index >= from (and < limit) in a bit array, or -1.
-__device__ __forceinline__ int next_bit(const uint32_t *bits, int from, int limit)
-{
-    if (from >= limit) return -1;
-    int w = from >> 5;
-    uint32_t word = bits[w] & (0xFFFFFFFFu << (from & 31));
-    const int nw = (limit + 31) >> 5;
-    for (;;) {
-        if (word) {
-            const int r = (w << 5) + __ffs(word) - 1;
-            return r < limit ? r : -1;
-        }
-        if (++w >= nw) return -1;
-        word = bits[w];
-    }
-}
-
-// The work-item sequence every role walks identically: correction chunks, then kept blocks.
+// The work-item sequence every role walks identically: the correction chunks whose bit is set in
+// `need`, then the key blocks whose bit is set in `mask_u`, each in ascending order.  The current
+// 32-bit mask word is kept in a register and its visited bits cleared, so a step is usually one
+// find-first-set (a step that re-scans shared memory cost about 450 cycles per item).
 struct Walker {
-    int phase = 0;   // 0: correction chunks, 1: kept blocks, 2: done
-    int idx = -1;
+    int phase = 0;      // 0: correction chunks, 1: kept blocks, 2: done
+    int idx = -1;       // the current item's chunk or block index
+    int wi = -1;        // index of the cached mask word
+    uint32_t cur = 0;   // its bits not yet visited
     __device__ __forceinline__ bool next(const Misc &m, const Params &p)
     {
-        if (phase == 0) {
-            const int c = next_bit(m.need, idx + 1, p.nchunks);
-            if (c >= 0) { idx = c; return true; }
-            phase = 1;
+        while (phase < 2) {
+            const uint32_t *bits = phase == 0 ? m.need : m.mask_u;
+            const int limit = phase == 0 ? p.nchunks : p.Nk;
+            const int nw = (limit + 31) >> 5;
+            while (cur == 0u && wi + 1 < nw) cur = bits[++wi];
+            if (cur != 0u) {
+                const int r = (wi << 5) + __ffs(cur) - 1;
+                cur &= cur - 1u;
+                if (r < limit) {   // bits past the limit are never set; the test is a safeguard
+                    idx = r;
+                    return true;
+                }
+            }
+            ++phase;
             idx = -1;
-        }
-        if (phase == 1) {
-            const int j = next_bit(m.mask_u, idx + 1, p.Nk);
-            if (j >= 0) { idx = j; return true; }
-            phase = 2;
+            wi = -1;
+            cur = 0u;
         }
         return false;
     }
@@ -255,7 +255,8 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
     for (int it = 0; ok && (more_k || more_v); ++it) {
         if (more_k) {
             const int s = it & 1;
-            if (it >= 2 && !wait_bar(&m.s_full[s], ((it - 2) >> 1) & 1, m, p, kSiteProdK)) { ok = false; break; }
+            constexpr int B = Geo<D>::kSBufs;
+            if (it >= 2 && !wait_bar(&m.s_full[(it - 2) % B], ((it - 2) / B) & 1, m, p, kSiteProdK)) { ok = false; break; }
             load_tile<D>(smem + G::kOffK + s * G::kKVTileBytes, wk.phase == 0 ? tm_kb : tm_k, &m.k_full[s], wk.idx * kTile, bh);
             issued_k[s] = it;
             more_k = wk.next(m, p);
@@ -280,21 +281,21 @@ template <int D>
 __device__ __forceinline__ bool issue_pv(int t, uint32_t tmem, uint64_t dv0, Misc &m, const Params &p)
 {
     using G = Geo<D>;
-    const int b = t & 1, s = t & 1;
-    const uint32_t ph = (t >> 1) & 1;
-    if (!wait_bar(&m.p_full[b], ph, m, p, kSiteMmaP)) return false;
-    if (!wait_bar(&m.v_full[s], ph, m, p, kSiteMmaV)) return false;
+    const int b = t % G::kSBufs, s = t & 1;
+    if (!wait_bar(&m.p_full[b], (t / G::kSBufs) & 1, m, p, kSiteMmaP)) return false;
+    if (!wait_bar(&m.v_full[s], (t >> 1) & 1, m, p, kSiteMmaV)) return false;
     tc_fence_after();
     // B = V tile of stage s, MN-major: 64 channels contiguous per key row (128 B, swizzled), next
     // 8 keys at +1024 B (SBO), channels 64..127 (d = 128) at +8192 B (LBO); 16 keys per MMA ->
     // +2048 B, i.e. +128 in the descriptor's 16-byte address units.
     const uint64_t dv = dv0 + static_cast<uint64_t>(s) * (G::kKVTileBytes >> 4);
     const uint32_t a0 = tmem + tmem_s_col(b);
-    if (t > 0) mma_ts_acc(tmem + kTmemO, a0, dv, G::kIdescPV);
-    else mma_ts(tmem + kTmemO, a0, dv, G::kIdescPV, 0u);
-    mma_ts_acc(tmem + kTmemO, a0 + 8, dv + 128, G::kIdescPV);
-    mma_ts_acc(tmem + kTmemO, a0 + 16, dv + 256, G::kIdescPV);
-    mma_ts_acc(tmem + kTmemO, a0 + 24, dv + 384, G::kIdescPV);
+    const uint32_t o = tmem + G::kTmemO;
+    if (t > 0) mma_ts_acc(o, a0, dv, G::kIdescPV);
+    else mma_ts(o, a0, dv, G::kIdescPV, 0u);
+    mma_ts_acc(o, a0 + 8, dv + 128, G::kIdescPV);
+    mma_ts_acc(o, a0 + 16, dv + 256, G::kIdescPV);
+    mma_ts_acc(o, a0 + 24, dv + 384, G::kIdescPV);
     mma_commit(&m.v_empty[s]);
     return true;
 }
@@ -317,10 +318,13 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
         const uint64_t dk0 = desc_sw128(smem_u32(smem + G::kOffK), 16, 1024);
         const uint64_t dv0 = desc_sw128(smem_u32(smem + G::kOffV), kKVHalfBytes, 1024);
         constexpr uint64_t kQh = kQHalfBytes >> 4, kKh = kKVHalfBytes >> 4;
+        // QK(it) is issued before PV(it - L), L = kSBufs - 1: S buffer it % kSBufs held P(it - kSBufs),
+        // whose PV was issued in an earlier iteration.
+        constexpr int L = G::kSBufs - 1;
         Walker w;
         int it = 0;
         while (ok && w.next(m, p)) {
-            const int s = it & 1, b = it & 1;
+            const int s = it & 1, b = it % G::kSBufs;
             if (!wait_bar(&m.k_full[s], (it >> 1) & 1, m, p, kSiteMmaK)) { ok = false; break; }
             tc_fence_after();
             const uint64_t dk = dk0 + static_cast<uint64_t>(s) * (G::kKVTileBytes >> 4);
@@ -336,14 +340,142 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
                 mma_ss_acc(d, dq + kQh + 6, dk + kKh + 6, G::kIdescQK);
             }
             mma_commit(&m.s_full[b]);
-            if (it > 0 && !issue_pv<D>(it - 1, tmem, dv0, m, p)) { ok = false; break; }
+            if (it >= L && !issue_pv<D>(it - L, tmem, dv0, m, p)) { ok = false; break; }
             ++it;
         }
-        if (ok && it > 0 && issue_pv<D>(it - 1, tmem, dv0, m, p)) mma_commit(&m.o_final);
+        for (int t = it - L < 0 ? 0 : it - L; ok && t < it; ++t) ok = issue_pv<D>(t, tmem, dv0, m, p);
+        if (ok && it > 0) mma_commit(&m.o_final);
     }
     // Every MMA issued so far must finish before TMEM is freed.
     mma_commit(&m.drain);
     wait_bar(&m.drain, 0, m, p, kSiteDrain, false);
+}
+
+// Kinds of softmax work item: a correction chunk of 64 pooled blocks, a full kept key block, and
+// the last key block when it is partial.  They run in separate loops (correction chunks first,
+// the partial block last), so the loop over full kept blocks, where the time goes, carries neither
+// the correction nor the tail-masking code (the smaller loop measured about 10 % faster per item).
+enum ItemKind : int { kItemCorr = 0, kItemFull = 1, kItemPartial = 2 };
+
+// One softmax work item for the thread that owns TMEM lane `row`: wait for S, mask, update the
+// running max (rescaling O in TMEM when it grows by more than 2^8), exponentiate, publish P.
+// Returns false if a wait gave up.
+template <int D, int kKind>
+__device__ __forceinline__ bool softmax_item(uint32_t tmem, Misc &m, const Params &p,
+                                             const uint32_t *mymask, uint32_t lane_base, int it,
+                                             int idx, float &m_used, float &l)
+{
+    const int b = it % Geo<D>::kSBufs;
+    bool ok = wait_bar(&m.s_full[b], (it / Geo<D>::kSBufs) & 1, m, p, kSiteSoftS);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (!ok) return false;
+    tc_fence_after();
+    const uint32_t s_addr = tmem + lane_base + tmem_s_col(b);
+    uint32_t pk[32];
+    bool rescale = false;
+    float factor = 1.0f;
+    const bool participate =
+        kKind == kItemCorr || ((mymask[idx >> 5] >> (idx & 31)) & 1u);   // warp-uniform
+    if (participate) {
+        uint32_t r[64];
+        tmem_ld64(s_addr, r);
+        tmem_wait_ld();
+        float mx;          // row max of the log2-domain logits of this item
+        uint64_t mul2;     // exp2 argument = r * mul2 - m_ref, two columns at a time
+        if constexpr (kKind == kItemCorr) {
+            // Correction chunk: column i is pooled block j0 + i with logit
+            // S*log2(e)/sqrt(d) + log2(n_j), or -inf if this row's tile kept block j (it is
+            // computed exactly) or j is past the last block.
+            const int c = idx;
+            const int j0 = c * 64;
+            uint64_t use = ~(static_cast<uint64_t>(mymask[2 * c]) |
+                             (static_cast<uint64_t>(mymask[2 * c + 1]) << 32));
+            const int nvalid = p.Nk - j0;
+            if (nvalid < 64) use &= (1ull << nvalid) - 1ull;
+            const int last = p.Nk - 1 - j0;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float bias = (i == last) ? p.last_bias_log2 : 6.0f;
+                const float x = fmaf(__uint_as_float(r[i]), p.scale_log2, bias);
+                r[i] = ((use >> i) & 1ull) ? __float_as_uint(x) : __float_as_uint(-INFINITY);
+            }
+            mul2 = f2(1.0f, 1.0f);
+        } else {
+            // Kept block: exact logits; columns past the sequence end (only in the last, partial
+            // block) are -inf.
+            if constexpr (kKind == kItemPartial) {
+                const int nvalid = p.N - idx * kTile;
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (i >= nvalid) r[i] = __float_as_uint(-INFINITY);
+            }
+            mul2 = f2(p.scale_log2, p.scale_log2);
+        }
+        mx = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+#pragma unroll
+        for (int i = 3; i < 63; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+        mx = fmaxf(mx, __uint_as_float(r[63]));
+        if constexpr (kKind != kItemCorr) mx *= p.scale_log2;
+        const float m_new = fmaxf(m_used, mx);
+        if (m_new > m_used + kRescaleLog2) {
+            factor = ex2_approx(m_used - m_new);
+            rescale = m_used != -INFINITY;
+            m_used = m_new;
+        }
+        const float mref = m_used == -INFINITY ? 0.0f : m_used;
+        const uint64_t add2 = f2(-mref, -mref);
+        uint64_t sum2 = f2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const uint64_t a2 = ffma2(f2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), mul2, add2);
+            float e0, e1;
+            if (i < kPolyPairs) {
+                exp2_poly2(a2, e0, e1);
+            } else {
+                float a0, a1;
+                unf2(a2, a0, a1);
+                e0 = ex2_approx(a0);
+                e1 = ex2_approx(a1);
+            }
+            sum2 = fadd2(sum2, f2(e0, e1));
+            pk[i] = pack_bf16x2(e0, e1);
+        }
+        float s0, s1;
+        unf2(sum2, s0, s1);
+        l = l * factor + (s0 + s1);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+    }
+    if (__any_sync(0xFFFFFFFFu, rescale) && it > 0) {
+        // PV(it-1) must be done before O is touched; its completion is the phase
+        // (it-1)>>1 of v_empty[(it-1)&1].  Here PV(it-3) has completed (s_full for item it
+        // was committed after PV(it-kSBufs), it-3 at the latest, was issued) and PV(it+1)
+        // waits for this thread's p_full arrival, so that barrier is either one phase short
+        // or complete: the parity is unambiguous.
+        ok = wait_bar(&m.v_empty[(it - 1) & 1], ((it - 1) >> 1) & 1, m, p, kSiteSoftO);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) return false;
+        tc_fence_after();
+        const float f = rescale ? factor : 1.0f;
+#pragma unroll 1
+        for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
+            uint32_t o[32];
+            const uint32_t oaddr = tmem + lane_base + Geo<D>::kTmemO + ch * 32;
+            tmem_ld32(oaddr, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st32(oaddr, o);
+        }
+    }
+    tmem_st32(s_addr, pk);
+    tmem_wait_st();
+    tc_fence_before();
+    // one arrival per warp, after every lane's P stores have completed
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&m.p_full[b]);
+    return true;
 }
 
 // Softmax warps 0-3: thread r owns row r of the 128-row tile (TMEM lane r).
@@ -359,115 +491,19 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
     Walker w;
     int it = 0;
     bool ok = true;
-    while (w.next(m, p)) {
-        const int b = it & 1;
-        ok = wait_bar(&m.s_full[b], (it >> 1) & 1, m, p, kSiteSoftS);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t s_addr = tmem + lane_base + tmem_s_col(b);
-        uint32_t pk[32];
-        bool rescale = false;
-        float factor = 1.0f;
-        const bool participate =
-            w.phase == 0 || ((mymask[w.idx >> 5] >> (w.idx & 31)) & 1u);   // warp-uniform
-        if (participate) {
-            uint32_t r[64];
-            tmem_ld64(s_addr, r);
-            tmem_wait_ld();
-            float mx;          // row max of the log2-domain logits of this item
-            uint64_t mul2;     // exp2 argument = r * mul2 - m_ref, two columns at a time
-            if (w.phase == 0) {
-                // Correction chunk: column i is pooled block j0 + i with logit
-                // S*log2(e)/sqrt(d) + log2(n_j), or -inf if this row's tile kept block j (it is
-                // computed exactly) or j is past the last block.
-                const int c = w.idx;
-                const int j0 = c * 64;
-                uint64_t use = ~(static_cast<uint64_t>(mymask[2 * c]) |
-                                 (static_cast<uint64_t>(mymask[2 * c + 1]) << 32));
-                const int nvalid = p.Nk - j0;
-                if (nvalid < 64) use &= (1ull << nvalid) - 1ull;
-                const int last = p.Nk - 1 - j0;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float bias = (i == last) ? p.last_bias_log2 : 6.0f;
-                    const float x = fmaf(__uint_as_float(r[i]), p.scale_log2, bias);
-                    r[i] = ((use >> i) & 1ull) ? __float_as_uint(x) : __float_as_uint(-INFINITY);
-                }
-                mul2 = f2(1.0f, 1.0f);
-            } else {
-                // Kept block: exact logits; columns past the sequence end are -inf.
-                const int t0 = w.idx * kTile;
-                if (t0 + 64 > p.N) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (t0 + i >= p.N) r[i] = __float_as_uint(-INFINITY);
-                }
-                mul2 = f2(p.scale_log2, p.scale_log2);
-            }
-            mx = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
-#pragma unroll
-            for (int i = 3; i < 63; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-            mx = fmaxf(mx, __uint_as_float(r[63]));
-            if (w.phase != 0) mx *= p.scale_log2;
-            const float m_new = fmaxf(m_used, mx);
-            if (m_new > m_used + kRescaleLog2) {
-                factor = ex2_approx(m_used - m_new);
-                rescale = m_used != -INFINITY;
-                m_used = m_new;
-            }
-            const float mref = m_used == -INFINITY ? 0.0f : m_used;
-            const uint64_t add2 = f2(-mref, -mref);
-            uint64_t sum2 = f2(0.0f, 0.0f);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const uint64_t a2 = ffma2(f2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), mul2, add2);
-                float e0, e1;
-                if (i < kPolyPairs) {
-                    exp2_poly2(a2, e0, e1);
-                } else {
-                    float a0, a1;
-                    unf2(a2, a0, a1);
-                    e0 = ex2_approx(a0);
-                    e1 = ex2_approx(a1);
-                }
-                sum2 = fadd2(sum2, f2(e0, e1));
-                pk[i] = pack_bf16x2(e0, e1);
-            }
-            float s0, s1;
-            unf2(sum2, s0, s1);
-            l = l * factor + (s0 + s1);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) pk[i] = 0u;
-        }
-        if (__any_sync(0xFFFFFFFFu, rescale) && it > 0) {
-            // PV(it-1) must be done before O is touched; its completion is the phase
-            // (it-1)>>1 of v_empty[(it-1)&1].  Here PV(it-2) has completed (s_full for item it
-            // was committed after PV(it-2) was issued) and PV(it) waits for this thread's p_full
-            // arrival, so that barrier is either one phase short or complete: the parity is
-            // unambiguous.
-            ok = wait_bar(&m.v_empty[(it - 1) & 1], ((it - 1) >> 1) & 1, m, p, kSiteSoftO);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            const float f = rescale ? factor : 1.0f;
-#pragma unroll 1
-            for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
-                uint32_t o[32];
-                const uint32_t oaddr = tmem + lane_base + kTmemO + ch * 32;
-                tmem_ld32(oaddr, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                tmem_st32(oaddr, o);
-            }
-        }
-        tmem_st32(s_addr, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&m.p_full[b]);
-        ++it;
+    bool more = w.next(m, p);
+    for (; ok && more && w.phase == 0; more = w.next(m, p)) {
+        ok = softmax_item<D, kItemCorr>(tmem, m, p, mymask, lane_base, it, w.idx, m_used, l);
+        it += ok;
+    }
+    const int partial = p.N % kTile ? p.Nk - 1 : -1;   // the last block when it is partial
+    for (; ok && more && w.idx != partial; more = w.next(m, p)) {
+        ok = softmax_item<D, kItemFull>(tmem, m, p, mymask, lane_base, it, w.idx, m_used, l);
+        it += ok;
+    }
+    if (ok && more) {   // the partial last block is the last item when it is kept
+        ok = softmax_item<D, kItemPartial>(tmem, m, p, mymask, lane_base, it, w.idx, m_used, l);
+        it += ok;
     }
     if (!ok || it == 0) return;
     // o_final is single-use: at this point two PVs may still be outstanding (the QK of the last
@@ -484,7 +520,7 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
 #pragma unroll 1
     for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + kTmemO + ch * 32, o);
+        tmem_ld32(tmem + lane_base + Geo<D>::kTmemO + ch * 32, o);
         tmem_wait_ld();
         if (store) {
 #pragma unroll
@@ -754,9 +790,9 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&m.v_full[s], 1);
             mbar_init(&m.v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kMaxSBufs; ++b) {
             mbar_init(&m.s_full[b], 1);
-            mbar_init(&m.p_full[b], kSoftmaxThreads);
+            mbar_init(&m.p_full[b], kSoftmaxThreads / 32);
         }
         mbar_init(&m.o_final, 1);
         mbar_init(&m.drain, 1);
