@@ -167,23 +167,31 @@ struct Params {
 
 __device__ __forceinline__ int volatile_load(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
 
-// Bounded wait on an mbarrier phase.  honor_abort=false is used while draining in-flight copies.
-__device__ bool wait_bar(uint64_t *bar, uint32_t parity, Misc &m, const Params &p, int site,
-                         bool honor_abort = true)
+// Slow path of wait_bar, out of line so that every wait site in the pipeline loops stays small.
+__device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, int *abort_flag,
+                                           DeviceStatus *status, unsigned long long timeout_ns,
+                                           int site, bool honor_abort)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15u) == 0) {
-            if (honor_abort && volatile_load(&m.abort_flag)) return false;
-            if (globaltimer_ns() - t0 > p.timeout_ns) {
-                *reinterpret_cast<volatile int *>(&m.abort_flag) = 1;
-                if (atomicCAS(&p.status->code, 0, 5) == 0) atomicExch(&p.status->where, site);
+            if (honor_abort && volatile_load(abort_flag)) return false;
+            if (globaltimer_ns() - t0 > timeout_ns) {
+                *reinterpret_cast<volatile int *>(abort_flag) = 1;
+                if (atomicCAS(&status->code, 0, 5) == 0) atomicExch(&status->where, site);
                 return false;
             }
         }
     }
+}
+
+// Bounded wait on an mbarrier phase.  honor_abort=false is used while draining in-flight copies.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Misc &m, const Params &p,
+                                         int site, bool honor_abort = true)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, &m.abort_flag, p.status, p.timeout_ns, site, honor_abort);
 }
 
 // The work-item sequence every role walks identically: the correction chunks whose bit is set in
