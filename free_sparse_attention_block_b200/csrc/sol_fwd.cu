@@ -203,11 +203,13 @@ struct Walker {
     int idx = -1;       // the current item's chunk or block index
     int wi = -1;        // index of the cached mask word
     uint32_t cur = 0;   // its bits not yet visited
-    __device__ __forceinline__ bool next(const Misc &m, const Params &p)
+    int nchunks, nblocks;   // bit counts of the two phases, held in registers
+    __device__ __forceinline__ explicit Walker(const Params &p) : nchunks(p.nchunks), nblocks(p.Nk) {}
+    __device__ __forceinline__ bool next(const Misc &m)
     {
         while (phase < 2) {
             const uint32_t *bits = phase == 0 ? m.need : m.mask_u;
-            const int limit = phase == 0 ? p.nchunks : p.Nk;
+            const int limit = phase == 0 ? nchunks : nblocks;
             const int nw = (limit + 31) >> 5;
             while (cur == 0u && wi + 1 < nw) cur = bits[++wi];
             if (cur != 0u) {
@@ -250,15 +252,15 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, 
 // phase of s_full[s] for that item (the S buffer and the K stage share the index); that phase
 // cannot be overtaken because QK(it) needs the tile loaded here.
 template <int D>
-__device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+__device__ __forceinline__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                               const CUtensorMap *tm_kb, const CUtensorMap *tm_vb, uint8_t *smem,
                               Misc &m, const Params &p, int bh)
 {
     using G = Geo<D>;
     int issued_k[kStages], issued_v[kStages];
     for (int s = 0; s < kStages; ++s) issued_k[s] = issued_v[s] = -1;
-    Walker wk, wv;
-    bool more_k = wk.next(m, p), more_v = wv.next(m, p);
+    Walker wk(p), wv(p);
+    bool more_k = wk.next(m), more_v = wv.next(m);
     bool ok = true;
     for (int it = 0; ok && (more_k || more_v); ++it) {
         if (more_k) {
@@ -267,7 +269,7 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
             if (it >= 2 && !wait_bar(&m.s_full[(it - 2) % B], ((it - 2) / B) & 1, m, p, kSiteProdK)) { ok = false; break; }
             load_tile<D>(smem + G::kOffK + s * G::kKVTileBytes, wk.phase == 0 ? tm_kb : tm_k, &m.k_full[s], wk.idx * kTile, bh);
             issued_k[s] = it;
-            more_k = wk.next(m, p);
+            more_k = wk.next(m);
         }
         const int iv = it - 1;
         if (iv >= 0 && more_v) {
@@ -275,7 +277,7 @@ __device__ void producer_role(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
             if (iv >= 2 && !wait_bar(&m.v_empty[s], ((iv - 2) >> 1) & 1, m, p, kSiteProdV)) { ok = false; break; }
             load_tile<D>(smem + G::kOffV + s * G::kKVTileBytes, wv.phase == 0 ? tm_vb : tm_v, &m.v_full[s], wv.idx * kTile, bh);
             issued_v[s] = iv;
-            more_v = wv.next(m, p);
+            more_v = wv.next(m);
         }
     }
     // No TMA write may still be in flight when the CTA exits.
@@ -309,7 +311,7 @@ __device__ __forceinline__ bool issue_pv(int t, uint32_t tmem, uint64_t dv0, Mis
 }
 
 template <int D>
-__device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
+__device__ __forceinline__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
 {
     using G = Geo<D>;
     bool ok = true;
@@ -329,9 +331,9 @@ __device__ void mma_role(uint32_t tmem, uint8_t *smem, Misc &m, const Params &p)
         // QK(it) is issued before PV(it - L), L = kSBufs - 1: S buffer it % kSBufs held P(it - kSBufs),
         // whose PV was issued in an earlier iteration.
         constexpr int L = G::kSBufs - 1;
-        Walker w;
+        Walker w(p);
         int it = 0;
-        while (ok && w.next(m, p)) {
+        while (ok && w.next(m)) {
             const int s = it & 1, b = it % G::kSBufs;
             if (!wait_bar(&m.k_full[s], (it >> 1) & 1, m, p, kSiteMmaK)) { ok = false; break; }
             tc_fence_after();
@@ -488,7 +490,7 @@ __device__ __forceinline__ bool softmax_item(uint32_t tmem, Misc &m, const Param
 
 // Softmax warps 0-3: thread r owns row r of the 128-row tile (TMEM lane r).
 template <int D>
-__device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, int row0)
+__device__ __forceinline__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, int row0)
 {
     const int row = threadIdx.x;                       // 0..127 == TMEM lane
     const int warp = row >> 5;
@@ -496,16 +498,16 @@ __device__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, in
     const uint32_t *mymask = in_b ? m.mask_b : m.mask_a;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     float m_used = -INFINITY, l = 0.0f;
-    Walker w;
+    Walker w(p);
     int it = 0;
     bool ok = true;
-    bool more = w.next(m, p);
-    for (; ok && more && w.phase == 0; more = w.next(m, p)) {
+    bool more = w.next(m);
+    for (; ok && more && w.phase == 0; more = w.next(m)) {
         ok = softmax_item<D, kItemCorr>(tmem, m, p, mymask, lane_base, it, w.idx, m_used, l);
         it += ok;
     }
     const int partial = p.N % kTile ? p.Nk - 1 : -1;   // the last block when it is partial
-    for (; ok && more && w.idx != partial; more = w.next(m, p)) {
+    for (; ok && more && w.idx != partial; more = w.next(m)) {
         ok = softmax_item<D, kItemFull>(tmem, m, p, mymask, lane_base, it, w.idx, m_used, l);
         it += ok;
     }
@@ -779,7 +781,10 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 {
     using G = Geo<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned by pointer arithmetic on the shared array, so that the compiler keeps
+    // everything derived from it in the shared address space (an integer round trip would make
+    // every Misc, mask and proxy-row access a generic one)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc &m = *reinterpret_cast<Misc *>(smem + G::kOffMisc);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pair = blockIdx.x % p.npairs;
