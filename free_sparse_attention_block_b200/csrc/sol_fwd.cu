@@ -40,6 +40,8 @@
 #include <cstddef>
 #include <mutex>
 
+#include <type_traits>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -421,34 +423,65 @@ __device__ __forceinline__ bool softmax_item(uint32_t tmem, Misc &m, const Param
             }
             mul2 = f2(p.scale_log2, p.scale_log2);
         }
-        mx = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+        uint64_t sum2;
+        // Exponentials against mref: P into pk, the row sum into sum2; with kTrack the pass also
+        // forms the item's row max (of r) in mx.
+        auto exp_pass = [&](float mref, auto track) {
+            constexpr bool kTrack = decltype(track)::value;
+            const uint64_t add2 = f2(-mref, -mref);
+            sum2 = f2(0.0f, 0.0f);
+            if constexpr (kTrack) mx = -INFINITY;
 #pragma unroll
-        for (int i = 3; i < 63; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-        mx = fmaxf(mx, __uint_as_float(r[63]));
-        if constexpr (kKind != kItemCorr) mx *= p.scale_log2;
-        const float m_new = fmaxf(m_used, mx);
-        if (m_new > m_used + kRescaleLog2) {
-            factor = ex2_approx(m_used - m_new);
-            rescale = m_used != -INFINITY;
-            m_used = m_new;
-        }
-        const float mref = m_used == -INFINITY ? 0.0f : m_used;
-        const uint64_t add2 = f2(-mref, -mref);
-        uint64_t sum2 = f2(0.0f, 0.0f);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const uint64_t a2 = ffma2(f2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), mul2, add2);
-            float e0, e1;
-            if (i < kPolyPairs) {
-                exp2_poly2(a2, e0, e1);
-            } else {
-                float a0, a1;
-                unf2(a2, a0, a1);
-                e0 = ex2_approx(a0);
-                e1 = ex2_approx(a1);
+            for (int i = 0; i < 32; ++i) {
+                const float r0 = __uint_as_float(r[2 * i]), r1 = __uint_as_float(r[2 * i + 1]);
+                if constexpr (kTrack) mx = max3f(mx, r0, r1);
+                const uint64_t a2 = ffma2(f2(r0, r1), mul2, add2);
+                float e0, e1;
+                if (i < kPolyPairs) {
+                    exp2_poly2(a2, e0, e1);
+                } else {
+                    float a0, a1;
+                    unf2(a2, a0, a1);
+                    e0 = ex2_approx(a0);
+                    e1 = ex2_approx(a1);
+                }
+                sum2 = fadd2(sum2, f2(e0, e1));
+                pk[i] = pack_bf16x2(e0, e1);
             }
-            sum2 = fadd2(sum2, f2(e0, e1));
-            pk[i] = pack_bf16x2(e0, e1);
+        };
+        if constexpr (Geo<D>::kSBufs >= 3) {
+            // With three S buffers the MMA warp runs two items ahead and the softmax is the
+            // critical path: the exponentials are taken against the running max m_used (which
+            // only moves when the item's max exceeds it by more than 2^8) while the item's max
+            // is formed in the same pass, so they do not wait for it.  When it moves (always on
+            // a row's first item, where m_used is -inf) the row repeats the pass against the new
+            // max; S stays in registers meanwhile.  The decisions and arguments are those of the
+            // max-first order below, so the results are identical.
+            float mref = m_used == -INFINITY ? 0.0f : m_used;
+            for (;;) {
+                exp_pass(mref, std::true_type{});
+                if constexpr (kKind != kItemCorr) mx *= p.scale_log2;
+                if (!(mx > m_used + kRescaleLog2)) break;
+                factor = ex2_approx(m_used - mx);
+                rescale = m_used != -INFINITY;
+                m_used = mx;
+                mref = mx;
+            }
+        } else {
+            // Max first.  With two S buffers the item chain through the MMA warp is the critical
+            // path, and the single-pass order above measured slower here.
+            mx = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+#pragma unroll
+            for (int i = 3; i < 63; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            mx = fmaxf(mx, __uint_as_float(r[63]));
+            if constexpr (kKind != kItemCorr) mx *= p.scale_log2;
+            const float m_new = fmaxf(m_used, mx);
+            if (m_new > m_used + kRescaleLog2) {
+                factor = ex2_approx(m_used - m_new);
+                rescale = m_used != -INFINITY;
+                m_used = m_new;
+            }
+            exp_pass(m_used == -INFINITY ? 0.0f : m_used, std::false_type{});
         }
         float s0, s1;
         unf2(sum2, s0, s1);
@@ -850,7 +883,10 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int c = tid, half = c >> 6, cc = c & 63, chunk = cc >> 3, within = cc & 7;
             const uint8_t *qh = smem + G::kOffQ + half * kQHalfBytes + within * 2;
             float sa = 0.0f, sb = 0.0f;
+            // unrolled so that the shared-memory loads run ahead of the (ordered) additions
+#pragma unroll 8
             for (int r = 0; r < n_a; ++r) sa += bf16_at(qh + r * 128 + ((chunk ^ (r & 7)) << 4));
+#pragma unroll 8
             for (int r = 0; r < n_b; ++r) {
                 const int rr = kTile + r;
                 sb += bf16_at(qh + rr * 128 + ((chunk ^ (rr & 7)) << 4));
