@@ -330,7 +330,9 @@ def config_of(wl, args):
     return {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "grid": list(wl.grid),
             "beta": args.beta, "tile": 64,
             "l2": "flushed before every timed step (256 MiB write)",
-            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+            "parallelism": ("single GPU" if args.gpus == 1 else
+                            f"head-sharded x{args.gpus}, outputs all-gathered" if args.shard == "heads"
+                            else f"replicas x{args.gpus}")}
 
 
 def run_ours(args, wl):
@@ -350,7 +352,17 @@ def run_ours(args, wl):
     torch.cuda.set_device(dev)
     sol.load_library()
 
-    q, k, v = inputs.gen_workload(wl)
+    shard = args.shard == "heads"
+    if shard:
+        # this rank's contiguous head range; the outputs are all-gathered inside every step
+        from free_sparse_attention_block_b200.sharded import gather_heads, head_range
+        h0, h1 = head_range(wl.H, rank, world)
+        if h1 == h0:
+            raise SystemExit(f"--shard heads: {wl.H} heads over {world} ranks leaves rank {rank} idle")
+        q, k, v = inputs.gen_workload(wl, heads=[(b, h) for b in range(wl.B) for h in range(h0, h1)])
+        q, k, v = (np.ascontiguousarray(x[:, h0:h1]) for x in (q, k, v))
+    else:
+        q, k, v = inputs.gen_workload(wl)
     B, H, N, d = q.shape
     Nq = wl.nq
     to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -379,6 +391,11 @@ def run_ours(args, wl):
         sol.sol_attn_fwd(tq, tk, tv, args.beta, ws, out, dens)
         if ev is not None:
             ev[2].record(stream)
+        if shard and world > 1:
+            gather_heads(out, wl.H)        # NCCL; the current stream waits for it
+            gather_heads(dens, wl.H)
+        if ev is not None:
+            ev[3].record(stream)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -388,7 +405,7 @@ def run_ours(args, wl):
     if st != 0:
         raise RuntimeError(f"device status {sol.STATUS.get(st)} at wait site {where}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -402,7 +419,8 @@ def run_ours(args, wl):
         dist.barrier()
     pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
     fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    step_ms = float(np.mean([a + b for a, b in zip(pool_ms, fwd_ms)]))
+    gather_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    step_ms = float(np.mean([e[0].elapsed_time(e[3]) for e in evs]))
     mean_fwd = float(np.mean(fwd_ms))
     mean_pool = float(np.mean(pool_ms))
     st, where = sol.sol_attn_read_status(ws)
@@ -412,7 +430,8 @@ def run_ours(args, wl):
     # max over ranks of the device time
     t_max = max_over_ranks(step_ms, dev)
     dense = wl.dense_flops()
-    value = replica_throughput(dense, world, t_max)
+    # replicas: every rank runs the whole workload; head-sharded: the ranks split one workload
+    value = dense / (t_max * 1e-3) / 1e12 if shard else replica_throughput(dense, world, t_max)
 
     # ---- e2e through the C ABI on pinned host buffers (copies inside the timed region)
     hq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -431,6 +450,7 @@ def run_ours(args, wl):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    e2e_value = dense / (e2e_ms * 1e-3) / 1e12 if shard else replica_throughput(dense, world, e2e_ms)
     assert torch.isfinite(hout.float()).all()
     h2d = 3 * B * H * N * d * 2
     d2h = B * H * N * d * 2 + B * H * Nq * 4
@@ -486,9 +506,11 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_of(wl, args) | {"seed": wl.seed},
         "fwd_ms": mean_fwd, "pool_ms": mean_pool,
+        "gather_ms": gather_ms if shard and world > 1 else None,
+        "heads_this_rank": int(H),
         "pool_gbs": (2 * B * H * N * d * 2 + B * H * Nq * d * 12) / (mean_pool * 1e-3) / 1e9,
         "density": fc["density"],
         "density_tokens": fc["density_tokens"],
@@ -501,7 +523,7 @@ def run_ours(args, wl):
                      "peak_source": f"bf16_tflops ({PEAK_SRC}; burst)", "kernel": "sol_fwd_kernel",
                      "algorithmic_flops_per_launch": fc["kept"] + fc["corr"]},
         "cpu_baseline": cpu,
-        "e2e": {"value": replica_throughput(dense, world, e2e_ms), "unit": UNIT, "ms": e2e_ms,
+        "e2e": {"value": e2e_value, "unit": UNIT, "ms": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "sol_attn_fwd_host (pinned host buffers)"},
         "gpu_launches": 2 * args.steps,
@@ -524,6 +546,9 @@ PEAK_BF16_SUST = float(PEAKS.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_t
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--shard", choices=["none", "heads"], default="none",
+                    help="with N > 1: split the workload's heads over the ranks and all-gather the "
+                         "outputs (strong scaling) instead of N independent replicas (weak)")
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
