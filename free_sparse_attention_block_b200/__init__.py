@@ -102,6 +102,50 @@ def _shape(t):
     return int(B), int(H), int(N), int(d)
 
 
+def _arg(name: str, t, dtype, shape=None, numel=None, cuda=True):
+    """Checks a tensor argument before its pointer reaches the library, which cannot see sizes:
+    dtype, exact shape or minimum element count, contiguity, then (unless cuda is None) the
+    device.  None and raw integer pointers pass unchecked (the caller vouches for them)."""
+    if t is None or isinstance(t, int):
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: needs at least {numel} elements, has {t.numel()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if cuda is not None and t.is_cuda != cuda:
+        raise ValueError(f"{name}: must be a {'CUDA' if cuda else 'host'} tensor")
+
+
+def _args(q, tensors: dict, workspace=None, density=None, host: dict | None = None,
+          host_density=None, debug: dict | None = None):
+    """Validates one call's tensors against q's [B, H, N, d]: every shape, dtype and size first,
+    then every device; returns (B, H, N, d)."""
+    import torch
+    B, H, N, d = _shape(q)
+    shp = (B, H, N, d)
+    Nq = (N + TILE - 1) // TILE
+    checks = [(name, t, torch.bfloat16, shp, None, True) for name, t in tensors.items()]
+    checks += [(name, t, torch.bfloat16, shp, None, False) for name, t in (host or {}).items()]
+    need = sol_attn_workspace_bytes(B, H, N, d)
+    if need:                     # 0: an unsupported shape, which the library itself reports
+        checks.append(("workspace", workspace, torch.uint8, None, need, True))
+    checks.append(("density", density, torch.int32, None, B * H * Nq, True))
+    checks.append(("host density", host_density, torch.int32, None, B * H * Nq, False))
+    if debug:
+        checks.append(("proxy_out", debug.get("proxy"), torch.float32, None, B * H * Nq * Nq, True))
+        checks.append(("mask_out", debug.get("mask"), torch.uint8, None, B * H * Nq * Nq, True))
+        checks.append(("stats_out", debug.get("stats"), torch.float32, None, B * H * Nq * 3, True))
+    for name, t, dtype, shape, numel, _ in checks:
+        _arg(name, t, dtype, shape=shape, numel=numel, cuda=None)
+    for name, t, dtype, shape, numel, cuda in checks:
+        _arg(name, t, dtype, shape=shape, numel=numel, cuda=cuda)
+    return shp
+
+
 def _check(status: int, where: str):
     if status != 0:
         raise SolError(status, where)
@@ -116,7 +160,7 @@ def sol_attn_workspace_bytes(B: int, H: int, N: int, d: int = HEAD_DIM) -> int:
 
 
 def sol_attn_pool(k, v, workspace, stream=None, check: bool = True) -> int:
-    B, H, N, d = _shape(k)
+    B, H, N, d = _args(k, {"k": k, "v": v}, workspace)
     st = load_library().sol_attn_pool(_ptr(k), _ptr(v), B, H, N, d, _ptr(workspace), _stream(stream))
     if check:
         _check(st, "sol_attn_pool")
@@ -125,7 +169,7 @@ def sol_attn_pool(k, v, workspace, stream=None, check: bool = True) -> int:
 
 def sol_attn_fwd(q, k, v, beta: float, workspace, out, density_out=None, stream=None,
                  check: bool = True) -> int:
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, workspace, density_out)
     st = load_library().sol_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(beta),
                                      _ptr(workspace), _ptr(out), _ptr(density_out), _stream(stream))
     if check:
@@ -136,9 +180,11 @@ def sol_attn_fwd(q, k, v, beta: float, workspace, out, density_out=None, stream=
 def sol_attn_fwd_betas(q, k, v, beta_per_head, workspace, out, density_out=None, stream=None,
                        check: bool = True) -> int:
     """sol_attn_fwd with one beta per head: beta_per_head is a float32 device tensor of B*H."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, workspace, density_out)
     if beta_per_head.numel() != B * H:
         raise ValueError("beta_per_head must hold B*H values")
+    import torch
+    _arg("beta_per_head", beta_per_head, torch.float32, numel=B * H)
     st = load_library().sol_attn_fwd_betas(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(beta_per_head),
                                            _ptr(workspace), _ptr(out), _ptr(density_out),
                                            _stream(stream))
@@ -150,7 +196,7 @@ def sol_attn_fwd_betas(q, k, v, beta_per_head, workspace, out, density_out=None,
 def sol_attn_fwd_topk(q, k, v, k_blocks: int, workspace, out, density_out=None, stream=None,
                       check: bool = True) -> int:
     """Forward with the top-k rule: the k_blocks highest-scoring blocks per query tile."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, workspace, density_out)
     st = load_library().sol_attn_fwd_topk(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(k_blocks),
                                           _ptr(workspace), _ptr(out), _ptr(density_out),
                                           _stream(stream))
@@ -163,7 +209,7 @@ def sol_attn_fwd_topp(q, k, v, p: float, workspace, out, density_out=None, strea
                       check: bool = True) -> int:
     """Forward with the top-p rule: the shortest highest-first prefix of blocks whose softmax
     probability over the proxy row reaches p."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, workspace, density_out)
     st = load_library().sol_attn_fwd_topp(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(p),
                                           _ptr(workspace), _ptr(out), _ptr(density_out),
                                           _stream(stream))
@@ -175,7 +221,8 @@ def sol_attn_fwd_topp(q, k, v, p: float, workspace, out, density_out=None, strea
 def sol_attn_fwd_debug_route(q, k, v, route, param: float, workspace, out, density_out=None,
                              proxy_out=None, mask_out=None, stats_out=None, stream=None) -> int:
     """Debug forward for any rule (``route``: a ROUTE name or code).  Returns the status code."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, workspace, density_out,
+                       debug={"proxy": proxy_out, "mask": mask_out, "stats": stats_out})
     code = ROUTE[route] if isinstance(route, str) else int(route)
     return load_library().sol_attn_fwd_debug_route(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, code, float(param), _ptr(workspace), _ptr(out),
@@ -186,7 +233,8 @@ def sol_attn_fwd_debug(q, k, v, beta: float, workspace, out, density_out=None, p
                        mask_out=None, stats_out=None, fault_flags: int = 0, timeout_ms: int = 0,
                        stream=None) -> int:
     """Returns the status code (it is not raised: tests inspect SOL_ERR_TIMEOUT)."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, workspace, density_out,
+                       debug={"proxy": proxy_out, "mask": mask_out, "stats": stats_out})
     return load_library().sol_attn_fwd_debug(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(beta), _ptr(workspace), _ptr(out),
         _ptr(density_out), _ptr(proxy_out), _ptr(mask_out), _ptr(stats_out), int(fault_flags),
@@ -201,7 +249,8 @@ def sol_attn_read_status(workspace, stream=None):
 
 def sol_attn_fwd_host(h_q, h_k, h_v, beta: float, d_q, d_k, d_v, workspace, d_out, h_out,
                       d_density=None, h_density=None, stream=None, check: bool = True) -> int:
-    B, H, N, d = _shape(d_q)
+    B, H, N, d = _args(d_q, {"d_q": d_q, "d_k": d_k, "d_v": d_v, "d_out": d_out}, workspace, d_density,
+                       host={"h_q": h_q, "h_k": h_k, "h_v": h_v, "h_out": h_out}, host_density=h_density)
     st = load_library().sol_attn_fwd_host(
         _ptr(h_q), _ptr(h_k), _ptr(h_v), B, H, N, d, float(beta), _ptr(d_q), _ptr(d_k), _ptr(d_v),
         _ptr(workspace), _ptr(d_out), _ptr(d_density), _ptr(h_out), _ptr(h_density), _stream(stream))
@@ -215,7 +264,7 @@ def sol_attn_fwd_noalloc(q, k, v, beta: float, out, density_out=None, stream=Non
     """Pool + forward without a caller workspace: the library's built-in scratch (at most
     NOALLOC_MAX_BYTES) holds the pooled keys/values.  For callers that cannot allocate device
     memory.  Calls that overlap on the GPU share that scratch and race; serialise them."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _args(q, {"q": q, "k": k, "v": v, "out": out}, density=density_out)
     st = load_library().sol_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(beta),
                                              _ptr(out), _ptr(density_out), _stream(stream))
     if check:
