@@ -279,7 +279,7 @@ def workspace_views(workspace, B: int, H: int, N: int, d: int = HEAD_DIM):
     Nk = (N + TILE - 1) // TILE
     n = B * H * Nk * d
     up = lambda x: (x + 255) & ~255
-    o_k32 = 256
+    o_k32 = 1024                       # after the header (status words, split counters)
     o_v32 = up(o_k32 + 4 * n)
     o_k16 = up(o_v32 + 4 * n)
     o_v16 = up(o_k16 + 2 * n)

@@ -13,7 +13,7 @@
 
 namespace sol {
 
-WorkspaceLayout workspace_layout(long long BH, long long Nk, int d)
+WorkspaceLayout workspace_layout(long long BH, long long Nk, int d, bool with_split)
 {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t elems = static_cast<size_t>(BH) * static_cast<size_t>(Nk) * static_cast<size_t>(d);
@@ -22,7 +22,10 @@ WorkspaceLayout workspace_layout(long long BH, long long Nk, int d)
     w.vbar32 = up(w.kbar32 + elems * 4);
     w.kbar16 = up(w.vbar32 + elems * 4);
     w.vbar16 = up(w.kbar16 + elems * 2);
-    w.total = up(w.vbar16 + elems * 2);
+    w.split_part = up(w.vbar16 + elems * 2);
+    const long long pairs = BH * ((Nk + 1) / 2);     // tile pairs of the call (Nq = Nk)
+    w.split_cap = with_split ? static_cast<int>(std::min<long long>(pairs, kSplitCap)) : 0;
+    w.total = up(w.split_part + static_cast<size_t>(w.split_cap) * 2 * kBM * (static_cast<size_t>(d) + 4) * 4);
     return w;
 }
 
@@ -106,11 +109,14 @@ struct Pooled {
     float *k32, *v32;
     uint8_t *k16, *v16;
     DeviceStatus *status;
+    int split_cap;       // the split region serves every head group of a call (one at a time)
+    int *split_cnt;
+    float *split_part;
 };
 
-Pooled pooled_at(void *workspace, const Shape &full, int bh0)
+Pooled pooled_at(void *workspace, const Shape &full, int bh0, bool with_split = true)
 {
-    const WorkspaceLayout wl = workspace_layout(full.BH, full.Nk, full.d);
+    const WorkspaceLayout wl = workspace_layout(full.BH, full.Nk, full.d, with_split);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const size_t off = static_cast<size_t>(bh0) * static_cast<size_t>(full.Nk) * static_cast<size_t>(full.d);
     Pooled p{};
@@ -119,8 +125,15 @@ Pooled pooled_at(void *workspace, const Shape &full, int bh0)
     p.k16 = ws + wl.kbar16 + off * 2;
     p.v16 = ws + wl.vbar16 + off * 2;
     p.status = reinterpret_cast<DeviceStatus *>(ws);
+    p.split_cap = wl.split_cap;
+    p.split_cnt = reinterpret_cast<int *>(ws + kSplitCntOffset);
+    p.split_part = reinterpret_cast<float *>(ws + wl.split_part);
     return p;
 }
+
+// Bytes at the start of the workspace that every call clears: the status words and the split
+// counters (the kernel also returns each counter it uses to zero).
+constexpr size_t kClearBytes = kSplitCntOffset + 4 * static_cast<size_t>(kSplitCap);
 
 // Pool K, V of the s.BH heads starting at k, v into `pw` (no argument checks).
 sol_status launch_pool(const void *k, const void *v, const Shape &s, const Pooled &pw, cudaStream_t stream)
@@ -165,6 +178,10 @@ sol_status launch_fwd(const void *q, const void *k, const void *v, const Shape &
     L.route = ra.route;
     L.topk = ra.topk;
     L.topp = ra.topp;
+    L.split_cap = pw.split_cap;
+    L.split_cnt = pw.split_cnt;
+    L.split_part = pw.split_part;
+    L.split_all = (fault_flags & 2) != 0;
     return launch_sol_fwd(L, stream) == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
 }
 
@@ -249,6 +266,28 @@ HostPipe *host_pipe()
 }
 
 }  // namespace
+
+// Pool + forward in a workspace laid out without the split region (the no-alloc entry point's
+// fixed scratch): the same kernels, no tile pair split over two CTAs.
+sol_status pool_fwd_unsplit(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                            float beta, void *workspace, void *out, int32_t *density, cudaStream_t stream)
+{
+    Shape s{};
+    sol_status st = check_shape(B, H, N, d, &s);
+    if (st != SOL_OK) return st;
+    if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
+    st = check_ptrs({q, k, v, workspace, out});
+    if (st != SOL_OK) return st;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
+    if (density && (reinterpret_cast<uintptr_t>(density) & 3u)) return SOL_ERR_ALIGNMENT;
+    if (cudaMemsetAsync(workspace, 0, kClearBytes, stream) != cudaSuccess) return SOL_ERR_CUDA;
+    const Pooled pw = pooled_at(workspace, s, 0, false);
+    st = launch_pool(k, v, s, pw, stream);
+    if (st != SOL_OK) return st;
+    return launch_fwd(q, k, v, s, pw, beta, nullptr, out, density, nullptr, nullptr, nullptr, 0,
+                      kDefaultTimeoutNs, stream, RouteArg{});
+}
+
 }  // namespace sol
 
 using namespace sol;
@@ -272,7 +311,7 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
     if (st != SOL_OK) return st;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), cs) != cudaSuccess) return SOL_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, kClearBytes, cs) != cudaSuccess) return SOL_ERR_CUDA;
     return launch_pool(k, v, s, pooled_at(workspace, s, 0), cs);
 }
 
@@ -392,7 +431,7 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
         std::max<size_t>(1, (upload + kHostGroupBytes - 1) / kHostGroupBytes)));
     const size_t head_dens = static_cast<size_t>(s.Nq) * sizeof(int32_t);
     auto fail = [](cudaError_t e) { return e != cudaSuccess; };
-    if (fail(cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), cs)) ||
+    if (fail(cudaMemsetAsync(workspace, 0, kClearBytes, cs)) ||
         fail(cudaEventRecord(hp->start, cs)) || fail(cudaStreamWaitEvent(hp->up, hp->start, 0)) ||
         fail(cudaStreamWaitEvent(hp->down, hp->start, 0)))
         return SOL_ERR_CUDA;

@@ -12,7 +12,11 @@ constexpr int kMaxHeadDim = 128;     // head dimensions d = 64 and d = 128 are c
 inline bool head_dim_supported(int d) { return d == 64 || d == 128; }
 constexpr int kTile = 64;            // query tile / key block length T
 constexpr int kMaxBlocks = 8192;     // Nk limit: two float proxy rows (64 KB) in shared memory
-constexpr size_t kHeaderBytes = 256; // workspace header (status words)
+constexpr size_t kHeaderBytes = 1024;  // workspace header: status words, then split counters
+constexpr size_t kSplitCntOffset = 256; // first split counter (int) in the header
+constexpr int kSplitCap = 128;          // most tile pairs one call splits over two CTAs
+static_assert(kSplitCntOffset + 4 * kSplitCap <= kHeaderBytes, "split counters fit the header");
+constexpr int kBM = 128;                // rows of one tile pair (two 64-row query tiles)
 
 // Device status words (first bytes of the workspace header).
 struct DeviceStatus {
@@ -20,11 +24,16 @@ struct DeviceStatus {
     int where;  // which wait gave up (see WaitSite in sol_fwd.cu)
 };
 
-// Workspace carve-up, all offsets in bytes from the workspace base.
+// Workspace carve-up, all offsets in bytes from the workspace base.  split_part holds, for up to
+// split_cap tile pairs processed by two CTAs each, both halves' unnormalised output rows with
+// their running max and sum: [split_cap][2][128 rows][d + 4] float32 (O[d], max, sum, 2 unused,
+// so every row starts 16-byte aligned).
 struct WorkspaceLayout {
-    size_t kbar32, vbar32, kbar16, vbar16, total;
+    size_t kbar32, vbar32, kbar16, vbar16, split_part, total;
+    int split_cap;
 };
-WorkspaceLayout workspace_layout(long long BH, long long Nk, int d);
+// with_split = false leaves out the split region (split_cap = 0: no tile pair is split).
+WorkspaceLayout workspace_layout(long long BH, long long Nk, int d, bool with_split = true);
 
 cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, int d, float *kbar32,
                            float *vbar32, void *kbar16, void *vbar16, cudaStream_t stream);
@@ -51,6 +60,10 @@ struct FwdLaunch {
     int route;      // Route
     int topk;       // kRouteTopK: blocks kept per query tile
     float topp;     // kRouteTopP: probability mass covered per query tile
+    int split_cap;  // tile pairs the workspace can split (0: none)
+    int *split_cnt;       // [split_cap] arrival counters, zero between calls
+    float *split_part;    // [split_cap][2][128][d + 4] partial rows
+    bool split_all;       // split every tile pair up to split_cap (test entry point)
 };
 cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream);
 

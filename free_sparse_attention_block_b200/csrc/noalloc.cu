@@ -32,12 +32,19 @@ sol_status shape_error(int B, int H, int N, int d)
 
 }  // namespace
 
+namespace sol {
+sol_status pool_fwd_unsplit(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                            float beta, void *workspace, void *out, int32_t *density, cudaStream_t stream);
+}
+
 extern "C" sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const void *v, int B,
                                            int H, int N, int d, float beta, void *out,
                                            int32_t *density_out, void *stream)
 {
-    const size_t need = sol_attn_workspace_bytes(B, H, N, d);
-    if (need == 0) return shape_error(B, H, N, d);
+    if (sol_attn_workspace_bytes(B, H, N, d) == 0) return shape_error(B, H, N, d);   // bad shape
+    const long long BH = static_cast<long long>(B) * H;
+    const long long Nk = (N + sol::kTile - 1) / sol::kTile;
+    const size_t need = sol::workspace_layout(BH, Nk, d, false).total;
     if (need > SOL_ATTN_NOALLOC_MAX_BYTES) return SOL_ERR_SCRATCH_LIMIT;
 
     int dev = 0;
@@ -47,9 +54,8 @@ extern "C" sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const v
     });
     if (g_err[dev] != cudaSuccess || g_addr[dev] == nullptr) return SOL_ERR_CUDA;
 
-    // sol_attn_pool clears the status words and overwrites every pooled row the forward reads,
-    // so nothing left in the array by an earlier call is used.
-    sol_status st = sol_attn_pool(k, v, B, H, N, d, g_addr[dev], stream);
-    if (st != SOL_OK) return st;
-    return sol_attn_fwd(q, k, v, B, H, N, d, beta, g_addr[dev], out, density_out, stream);
+    // The pool clears the status words and overwrites every pooled row the forward reads, so
+    // nothing left in the array by an earlier call is used.  The scratch has no split region.
+    return sol::pool_fwd_unsplit(q, k, v, B, H, N, d, beta, g_addr[dev], out, density_out,
+                                 static_cast<cudaStream_t>(stream));
 }

@@ -36,6 +36,7 @@
 // and MMAs land, frees its TMEM and exits.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstddef>
 #include <mutex>
@@ -53,7 +54,6 @@ constexpr int kNumWarps = 6;
 constexpr int kSoftmaxThreads = 128;   // warps 0-3: one thread per row (TMEM lane)
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
-constexpr int kBM = 128;
 
 constexpr uint32_t kQHalfBytes = kBM * 64 * 2;         // 128 rows x 64 channels, bf16
 constexpr uint32_t kKVHalfBytes = kTile * 64 * 2;      // 64 rows x 64 channels, bf16
@@ -111,7 +111,7 @@ enum SelState : int { kSelRun = 0, kSelNone = 1, kSelAll = 2 };
 enum WaitSite : int {
     kSiteQ = 1, kSiteProdK = 2, kSiteProdV = 3, kSiteMmaK = 4, kSiteMmaP = 5, kSiteMmaV = 6,
     kSiteSoftS = 7, kSiteSoftO = 8, kSiteEpilogue = 9, kSiteFault = 10, kSiteDrain = 11,
-    kSiteProdDrain = 12
+    kSiteProdDrain = 12, kSiteMerge = 13
 };
 
 struct Misc {
@@ -119,6 +119,7 @@ struct Misc {
     double mu[2], sigma[2], tau[2];
     uint64_t q_full, k_full[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[kMaxSBufs], p_full[kMaxSBufs], o_final, drain, never;
+    uint64_t merge_full;      // the other half's partial rows have landed (split units)
     uint32_t mask_a[kMaskWords];
     uint32_t mask_b[kMaskWords];
     uint32_t mask_u[kMaskWords];
@@ -137,6 +138,7 @@ struct Misc {
     uint32_t tmem_base;
     int abort_flag;
     int count_a, count_b;
+    int split_n, split_half, split_slot, split_old;   // split units (two CTAs)
 };
 
 template <int D>
@@ -165,6 +167,9 @@ struct Params {
     int route;               // kRouteThreshold, kRouteTopK or kRouteTopP
     int topk;                // blocks kept per query tile (top-k)
     float topp;              // probability mass to cover per query tile (top-p)
+    int split_first;         // units from this one on run as two CTAs each (the unit count: none)
+    int *split_cnt;          // arrival counter per split unit, zero between calls
+    float *split_part;       // [split unit][half][128 rows][D + 4] partial rows
 };
 
 __device__ __forceinline__ int volatile_load(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
@@ -521,6 +526,134 @@ __device__ __forceinline__ bool softmax_item(uint32_t tmem, Misc &m, const Param
     return true;
 }
 
+// Epilogue of a unit split over two CTAs; softmax threads, one per row (TMEM lane).  Each half
+// counts its arrival on the unit's counter.  The first to arrive writes its rows' unnormalised
+// output O (relative to 2^m), running max m (log2 domain) and sum l to its partial slot and counts
+// again; the second waits until the counter reads 3 (a bounded wait on a CTA that has already
+// arrived, so is running, and has nothing left to wait for), brings those rows into shared memory
+// and merges:
+//   out = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)),
+//   M = max(m_0, m_1),
+// the online-softmax combination of two disjoint sets of terms.  A half without items (has_o
+// false) contributes m = -inf, l = 0 and O = 0.  If any softmax warp's waits failed (ok false),
+// the CTA does not arrive (the other half then arrives first and publishes) and the status words
+// hold the timeout.
+template <int D>
+__device__ __forceinline__ void split_epilogue(uint32_t tmem, Misc &m, const Params &p, int bh, int row0,
+                                            uint32_t lane_base, bool ok, bool has_o, float m_used, float l)
+{
+    uint32_t all_ok;
+    asm volatile("{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\t"
+                 "bar.red.and.pred b, 1, %2, a;\n\tselp.u32 %0, 1, 0, b;\n\t}"
+                 : "=r"(all_ok)
+                 : "r"(static_cast<uint32_t>(ok)), "r"(kSoftmaxThreads)
+                 : "memory");
+    if (!all_ok) return;
+    constexpr int kRow = D + 4;   // floats per partial row: O[D], m, l, 2 unused (16-byte rows)
+    const int row = threadIdx.x;
+    const int slot = m.split_slot, half = m.split_half;
+    int *cnt = p.split_cnt + slot;
+    // Arrival first: the first half to arrive publishes its rows and counts again (the counter
+    // reaches 3 once both halves have arrived and the rows are out); the second merges and never
+    // writes its own partial rows.
+    if (row == 0) m.split_old = atomicAdd(cnt, 1);
+    asm volatile("bar.sync 1, %0;" ::"r"(kSoftmaxThreads) : "memory");
+    if (m.split_old == 0) {
+        float *mine = p.split_part + (static_cast<size_t>(2 * slot + half) * kBM + row) * kRow;
+#pragma unroll 1
+        for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
+            uint32_t o[32];
+            if (has_o) {
+                tmem_ld32(tmem + lane_base + Geo<D>::kTmemO + ch * 32, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = 0u;
+            }
+            float4 *dst = reinterpret_cast<float4 *>(mine + ch * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
+                                     __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
+        }
+        mine[D] = m_used;
+        mine[D + 1] = l;
+        __threadfence();                                           // the rows are visible ...
+        asm volatile("bar.sync 1, %0;" ::"r"(kSoftmaxThreads) : "memory");
+        if (row == 0) atomicAdd(cnt, 1);                           // ... before this count
+        return;
+    }
+    // Second: wait (bounded) until the first half's rows are out.  The first half has already
+    // arrived, so it is running and its publication ends.
+    if (row == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        int seen;
+        for (;;) {
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(cnt) : "memory");
+            if (seen >= 3) break;
+            if (globaltimer_ns() - t0 > p.timeout_ns) {
+                if (atomicCAS(&p.status->code, 0, 5) == 0) atomicExch(&p.status->where, kSiteMerge);
+                break;
+            }
+            __nanosleep(256);
+        }
+        m.split_old = seen >= 3 ? 1 : -1;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(kSoftmaxThreads) : "memory");
+    if (m.split_old < 0) return;
+    __threadfence();
+    // The other half's 128 rows are one contiguous block: one bulk copy brings them into shared
+    // memory (the Q tile and the K/V ring are idle: every MMA of this CTA has completed).
+    constexpr uint32_t kRowsBytes = kBM * kRow * 4;
+    static_assert(kRowsBytes <= Geo<D>::kOffMisc && kRowsBytes % 16 == 0, "partial rows fit the idle tiles");
+    float *rows = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(&m) - Geo<D>::kOffMisc);
+    if (row == 0) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(&m.merge_full, kRowsBytes);
+        bulk_load(rows, p.split_part + static_cast<size_t>(2 * slot + (half ^ 1)) * kBM * kRow, kRowsBytes,
+                  &m.merge_full);
+    }
+    if (!wait_bar(&m.merge_full, 0, m, p, kSiteMerge, false)) return;
+    const float *theirs = rows + row * kRow;
+    const float mo = theirs[D], lo = theirs[D + 1];
+    const float M = fmaxf(m_used, mo);
+    const float wa = m_used == -INFINITY ? 0.0f : ex2_approx(m_used - M);
+    const float wb = mo == -INFINITY ? 0.0f : ex2_approx(mo - M);
+    // half 0's term first whichever half merges, so the rounding (one fused multiply-add) and
+    // hence the output do not depend on which CTA finished second
+    auto sum2 = [&](float own_x, float own_w, float their_x, float their_w) {
+        return half == 0 ? fmaf(own_x, own_w, their_x * their_w) : fmaf(their_x, their_w, own_x * own_w);
+    };
+    const float inv = 1.0f / sum2(l, wa, lo, wb);
+    const int grow = row0 + row;
+    const bool store = grow < p.N;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + (store ? grow : 0)) * D);
+#pragma unroll 1
+    for (int ch = 0; ch < Geo<D>::kOChunks; ++ch) {
+        uint32_t o[32];
+        if (has_o) {
+            tmem_ld32(tmem + lane_base + Geo<D>::kTmemO + ch * 32, o);
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        const float4 *src = reinterpret_cast<const float4 *>(theirs + ch * 32);
+        auto mix = [&](int i, float t) { return sum2(__uint_as_float(o[i]), wa, t, wb) * inv; };
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 t0 = src[2 * q4], t1 = src[2 * q4 + 1];
+            uint4 w;
+            w.x = pack_bf16x2(mix(8 * q4 + 0, t0.x), mix(8 * q4 + 1, t0.y));
+            w.y = pack_bf16x2(mix(8 * q4 + 2, t0.z), mix(8 * q4 + 3, t0.w));
+            w.z = pack_bf16x2(mix(8 * q4 + 4, t1.x), mix(8 * q4 + 5, t1.y));
+            w.w = pack_bf16x2(mix(8 * q4 + 6, t1.z), mix(8 * q4 + 7, t1.w));
+            if (store) dst[ch * 4 + q4] = w;
+        }
+    }
+    if (row == 0) p.split_cnt[slot] = 0;   // ready for the next call
+}
+
 // Softmax warps 0-3: thread r owns row r of the 128-row tile (TMEM lane r).
 template <int D>
 __device__ __forceinline__ void softmax_role(uint32_t tmem, Misc &m, const Params &p, int bh, int row0)
@@ -548,10 +681,22 @@ __device__ __forceinline__ void softmax_role(uint32_t tmem, Misc &m, const Param
         ok = softmax_item<D, kItemPartial>(tmem, m, p, mymask, lane_base, it, w.idx, m_used, l);
         it += ok;
     }
-    if (!ok || it == 0) return;
     // o_final is single-use: at this point two PVs may still be outstanding (the QK of the last
     // item is issued before the PV of the one before it), so no per-stage parity identifies the
     // last PV.
+    if (m.split_n > 1) {
+        // Every softmax warp enters the split epilogue, whose barriers count all four, even after
+        // a failed wait (every wait is bounded, so every warp gets here).  Half of a unit may
+        // have no item.
+        if (ok && it > 0) {
+            ok = wait_bar(&m.o_final, 0, m, p, kSiteEpilogue);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (ok) tc_fence_after();
+        }
+        split_epilogue<D>(tmem, m, p, bh, row0, lane_base, ok, it > 0, m_used, l);
+        return;
+    }
+    if (!ok || it == 0) return;   // (a whole unit always has an item)
     ok = wait_bar(&m.o_final, 0, m, p, kSiteEpilogue);
     ok = __all_sync(0xFFFFFFFFu, ok);
     if (!ok) return;
@@ -804,6 +949,41 @@ __device__ __forceinline__ void load_vec(const float *src, float (&x)[LC])
     }
 }
 
+// One warp.  The walk visits the set bits of `need` (correction chunks) and then of `mask_u` (kept
+// blocks), each in ascending order; this keeps the items at even (half 0) or odd (half 1)
+// positions of the walk and clears the others, so every role of this CTA walks its half with the
+// ordinary walker.
+__device__ __forceinline__ void keep_half_of_walk(Misc &m, const Params &p, int half)
+{
+    const int lane = threadIdx.x & 31;
+    int parity = 0;   // walk position of the first set bit of the current group of words, mod 2
+    for (int phase = 0; phase < 2; ++phase) {
+        uint32_t *bits = phase == 0 ? m.need : m.mask_u;
+        const int nw = ((phase == 0 ? p.nchunks : p.Nk) + 31) >> 5;
+        for (int w0 = 0; w0 < nw; w0 += 32) {
+            const int w = w0 + lane;
+            const uint32_t x = w < nw ? bits[w] : 0u;
+            const int c = __popc(x);
+            int incl = c;   // inclusive prefix over the lanes of the set-bit counts
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int pos = parity + incl - c;
+            uint32_t keep = 0u, rest = x;
+            while (rest) {
+                const uint32_t b = rest & (0u - rest);
+                if ((pos & 1) == half) keep |= b;
+                rest ^= b;
+                ++pos;
+            }
+            if (w < nw) bits[w] = keep;
+            parity = (parity + __shfl_sync(0xFFFFFFFFu, incl, 31)) & 1;
+        }
+    }
+}
+
 // kRank: the top-k / top-p rules (radix selection) are compiled in; the threshold rule's kernel is
 // a separate instantiation without that code, which otherwise costs it about 3 % (measured).
 template <int D, bool kRank>
@@ -820,8 +1000,18 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc &m = *reinterpret_cast<Misc *>(smem + G::kOffMisc);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int pair = blockIdx.x % p.npairs;
-    const int bh = blockIdx.x / p.npairs;
+    // Work unit: a pair of query tiles of one head.  The units from split_first on run as two
+    // CTAs each (halves 0 and 1 on adjacent block indices), every other item of the unit's walk
+    // on each; the second to finish merges the two partial results.
+    int unit = blockIdx.x, split_n = 1, split_half = 0;
+    if (unit >= p.split_first) {
+        const int r = unit - p.split_first;
+        unit = p.split_first + (r >> 1);
+        split_half = r & 1;
+        split_n = 2;
+    }
+    const int pair = unit % p.npairs;
+    const int bh = unit / p.npairs;
     const int tile_a = 2 * pair, tile_b = 2 * pair + 1;
     const bool has_b = tile_b < p.Nq;
     const int row0 = tile_a * kTile;
@@ -841,11 +1031,15 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&m.p_full[b], kSoftmaxThreads / 32);
         }
         mbar_init(&m.o_final, 1);
+        mbar_init(&m.merge_full, 1);
         mbar_init(&m.drain, 1);
         mbar_init(&m.never, 1);
         m.abort_flag = 0;
         m.count_a = 0;
         m.count_b = 0;
+        m.split_n = split_n;
+        m.split_half = split_half;
+        m.split_slot = unit - p.split_first;
         fence_mbar_init();
     }
     for (int i = tid; i < kMaskWords; i += kThreads) {
@@ -1124,6 +1318,10 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (has_b) p.density[unit_a + 1] = m.count_b;
         }
     }
+    if (split_n > 1) {
+        __syncthreads();                          // need and mask_u are complete
+        if (warp == 0) keep_half_of_walk(m, p, split_half);
+    }
     fence_proxy_async_smem();   // generic writes to the ring happen-before the TMA overwrites it
     __syncthreads();
 
@@ -1149,10 +1347,24 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
+// Work units run as two CTAs each when they do not fill the last wave of CTAs (two resident per
+// SM): about 1.5 times the units of a last wave that is at most half full.  On the 12-head,
+// 16384-token call that splits 84 of 1536 units (56 past five full waves of 296): 1.9 % faster at
+// d = 128 and 3 % at d = 64, measured with the merge (without it, 84 to 150 split units were
+// equally good).  A fuller last wave, or a call of less than one wave, splits nothing.
+long long split_units(long long units, int slots, int cap)
+{
+    if (cap <= 0 || slots <= 0 || units <= slots) return 0;
+    const long long tail = units % slots;
+    if (tail == 0 || 2 * tail > slots) return 0;
+    return std::min<long long>(std::min<long long>(cap, units), tail + tail / 2);
+}
+
 template <int D, bool kRank>
 cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
 {
     static std::once_flag attr_once[64];
+    static int sm_count[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1162,6 +1374,8 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     std::call_once(attr_once[dev], [&] {
         attr_err = cudaFuncSetAttribute(sol_fwd_kernel<D, kRank>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(kSmem));
+        if (attr_err == cudaSuccess)
+            attr_err = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
     });
     if (attr_err != cudaSuccess) return attr_err;
 
@@ -1190,8 +1404,14 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     p.route = L.route;
     p.topk = L.topk;
     p.topp = L.topp;
-    const long long grid = static_cast<long long>(p.npairs) * L.BH;
-    if (grid <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const long long units = static_cast<long long>(p.npairs) * L.BH;
+    const long long S = L.split_all ? std::min<long long>(units, std::max(L.split_cap, 0))
+                                    : split_units(units, 2 * sm_count[dev], L.split_cap);
+    p.split_first = static_cast<int>(units - S);
+    p.split_cnt = L.split_cnt;
+    p.split_part = L.split_part;
+    const long long grid = units + S;
+    if (units <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     sol_fwd_kernel<D, kRank><<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(
         *L.tm_q, *L.tm_k, *L.tm_v, *L.tm_kb, *L.tm_vb, p);
     return cudaGetLastError();

@@ -55,9 +55,12 @@ typedef enum {
     SOL_ERR_SCRATCH_LIMIT = 6 /* sol_attn_fwd_noalloc: the shape needs more scratch than it has */
 } sol_status;
 
-/* Bytes of device workspace sol_attn_pool/sol_attn_fwd need for this shape: a 256-byte header
- * (status words) followed by the pooled keys and values, float32 [B,H,Nk,d] each, and their
- * bfloat16 copies [B,H,Nk,d] each.  Returns 0 for an invalid or unsupported shape. */
+/* Bytes of device workspace sol_attn_pool/sol_attn_fwd need for this shape: a 1 KB header
+ * (status words and the counters of split tile pairs), the pooled keys and values, float32
+ * [B,H,Nk,d] each, their bfloat16 copies [B,H,Nk,d] each, and room for the partial output rows
+ * of up to 128 tile pairs that the forward splits over two CTAs to fill its last wave of CTAs
+ * (2 x 128 rows x (d + 4) float32 per pair; 17 MB at d = 128 once the call has 128 tile pairs).
+ * Returns 0 for an invalid or unsupported shape. */
 size_t sol_attn_workspace_bytes(int B, int H, int N, int d);
 
 /* Mean-pool K and V into 64-token blocks (the k_bar_j / v_bar_j of the routing and of the
@@ -74,7 +77,12 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
  * online-softmax pass, and writes out = softmax-weighted values rounded to bfloat16.
  * beta: any non-NaN float, +-inf allowed.
  * density_out: device int32 [B,H,Nq], number of kept blocks per query tile, or NULL.
- * workspace: the one sol_attn_pool filled for this K, V (its status words may be written). */
+ * workspace: the one sol_attn_pool filled for this K, V (its status words may be written, and
+ * the split region is used as scratch; calls that share a workspace must not overlap on the GPU).
+ * Work unit: a pair of query tiles of one head per CTA.  When the units do not fill the last wave
+ * of CTAs (two per SM), the last units run as two CTAs each, every other item of the unit's work
+ * list on each; the second of the two to finish merges both partial rows (their own running max
+ * and sum) into the output.  The result is the same attention up to float rounding order. */
 sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
                         float beta, void *workspace, void *out, int32_t *density_out,
                         void *stream);
@@ -178,9 +186,12 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
  * packaging of the same two kernels.  Inputs and outputs are the caller's (as for sol_attn_fwd);
  * the pooled keys/values and status words go to a scratch array inside the library instead of a
  * caller workspace.  This entry point calls no cudaMalloc, cudaFree or other allocating routine.
- *   - Limit: sol_attn_workspace_bytes(B, H, N, d) <= SOL_ATTN_NOALLOC_MAX_BYTES, i.e.
- *     B*H*ceil(N/64) <= 10922 pooled rows at d = 128, 21845 at d = 64 (a 12-head, 16384-token
- *     call fits); larger shapes return SOL_ERR_SCRATCH_LIMIT without launching anything.
+ *   - Limit: the call's pooled keys and values (12 bytes per pooled channel) and a 1 KB header
+ *     fit in SOL_ATTN_NOALLOC_MAX_BYTES, i.e. B*H*ceil(N/64) <= 10922 pooled rows at d = 128,
+ *     21844 at d = 64 (a 12-head, 16384-token call fits); larger shapes return
+ *     SOL_ERR_SCRATCH_LIMIT without launching anything.  This entry point never splits a tile
+ *     pair over two CTAs (the scratch has no room for the partial rows), so its last wave of
+ *     CTAs may run less full than sol_attn_fwd's.
  *   - The first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any stream
  *     capture.

@@ -42,15 +42,24 @@ def test_workspace_bytes(lib):
     Nk = N // 64
     n = B * H * Nk * 128
     got = sol.sol_attn_workspace_bytes(B, H, N, 128)
-    assert got >= 256 + n * (4 + 4 + 2 + 2) and got % 256 == 0
-    assert sol.sol_attn_workspace_bytes(1, 1, 100, 128) > 0
+    up = lambda x: (x + 255) & ~255
+
+    def layout(BH, Nk, d):
+        # 1 KB header; float32 k_bar, v_bar; bf16 k_bar, v_bar; then the partial rows of up to
+        # 128 split tile pairs: [pairs][2 halves][128 rows][d + 4] float32
+        e = BH * Nk * d
+        pooled = up(up(up(up(1024 + 4 * e) + 4 * e) + 2 * e) + 2 * e)
+        cap = min(BH * ((Nk + 1) // 2), 128)
+        return up(pooled + cap * 2 * 128 * (d + 4) * 4)
+
+    assert got == layout(B * H, Nk, 128) and got % 256 == 0
+    assert got >= 1024 + n * (4 + 4 + 2 + 2) + 128 * 2 * 128 * 132 * 4       # 1536 pairs: cap 128
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 128) == layout(1, 2, 128)  # one pair: cap 1
     assert sol.sol_attn_workspace_bytes(1, 1, 100, 96) == 0       # d not 64/128: unsupported
     assert sol.sol_attn_workspace_bytes(1, 1, 100, 256) == 0
     # d = 64: the same layout with 64-channel rows
-    Nk64 = 2
-    n64 = 1 * 1 * Nk64 * 64
-    up = lambda x: (x + 255) & ~255
-    assert sol.sol_attn_workspace_bytes(1, 1, 100, 64) == up(up(up(up(256 + 4 * n64) + 4 * n64) + 2 * n64) + 2 * n64)
+    assert sol.sol_attn_workspace_bytes(1, 1, 100, 64) == layout(1, 2, 64)
+    assert sol.sol_attn_workspace_bytes(2, 3, 64 * 5 + 1, 64) == layout(6, 6, 64)
     assert sol.sol_attn_workspace_bytes(0, 1, 100, 128) == 0
     assert sol.sol_attn_workspace_bytes(1, 1, 524288 + 1, 128) == 0
 

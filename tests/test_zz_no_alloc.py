@@ -44,5 +44,8 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     # 12 heads x 65536 tokens needs 12 * 1024 pooled rows * 1536 B > 16 MiB
     st = lib.sol_attn_fwd_noalloc(A, A, A, 1, 12, 65536, 128, 0.5, A, None, None)
     assert sol.STATUS[st] == "SOL_ERR_SCRATCH_LIMIT"
-    assert sol.sol_attn_workspace_bytes(1, 12, 65536) > sol.NOALLOC_MAX_BYTES
-    assert sol.sol_attn_workspace_bytes(1, 12, 16384) <= sol.NOALLOC_MAX_BYTES
+    # the first row counts past the documented limits (10922 pooled rows at d = 128, 21844 at
+    # d = 64): 3 heads x 3641 blocks and 5 heads x 4369 blocks
+    for H, nblk, d in [(3, 3641, 128), (5, 4369, 64)]:
+        st = lib.sol_attn_fwd_noalloc(A, A, A, 1, H, 64 * nblk, d, 0.5, A, None, None)
+        assert sol.STATUS[st] == "SOL_ERR_SCRATCH_LIMIT", (H, nblk, d)
