@@ -112,6 +112,8 @@ struct Pooled {
     int split_cap;       // the split region serves every head group of a call (one at a time)
     int *split_cnt;
     float *split_part;
+    long long call_units;   // tile pairs of the whole call, and of the heads before bh0
+    long long unit0;
 };
 
 Pooled pooled_at(void *workspace, const Shape &full, int bh0, bool with_split = true)
@@ -128,6 +130,9 @@ Pooled pooled_at(void *workspace, const Shape &full, int bh0, bool with_split = 
     p.split_cap = wl.split_cap;
     p.split_cnt = reinterpret_cast<int *>(ws + kSplitCntOffset);
     p.split_part = reinterpret_cast<float *>(ws + wl.split_part);
+    const long long pairs = (full.Nq + 1) / 2;
+    p.call_units = static_cast<long long>(full.BH) * pairs;
+    p.unit0 = static_cast<long long>(bh0) * pairs;
     return p;
 }
 
@@ -182,6 +187,8 @@ sol_status launch_fwd(const void *q, const void *k, const void *v, const Shape &
     L.split_cnt = pw.split_cnt;
     L.split_part = pw.split_part;
     L.split_all = (fault_flags & 2) != 0;
+    L.call_units = pw.call_units;
+    L.unit0 = pw.unit0;
     return launch_sol_fwd(L, stream) == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
 }
 

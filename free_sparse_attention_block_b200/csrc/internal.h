@@ -64,6 +64,8 @@ struct FwdLaunch {
     int *split_cnt;       // [split_cap] arrival counters, zero between calls
     float *split_part;    // [split_cap][2][128][d + 4] partial rows
     bool split_all;       // split every tile pair up to split_cap (test entry point)
+    long long call_units; // tile pairs of the whole call this launch is part of (its head groups)
+    long long unit0;      // the call's index of this launch's first tile pair
 };
 cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream);
 

@@ -168,6 +168,7 @@ struct Params {
     int topk;                // blocks kept per query tile (top-k)
     float topp;              // probability mass to cover per query tile (top-p)
     int split_first;         // units from this one on run as two CTAs each (the unit count: none)
+    int split_slot0;         // the call's split slot of unit split_first (head groups of one call)
     int *split_cnt;          // arrival counter per split unit, zero between calls
     float *split_part;       // [split unit][half][128 rows][D + 4] partial rows
 };
@@ -1039,7 +1040,7 @@ sol_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         m.count_b = 0;
         m.split_n = split_n;
         m.split_half = split_half;
-        m.split_slot = unit - p.split_first;
+        m.split_slot = unit - p.split_first + p.split_slot0;
         fence_mbar_init();
     }
     for (int i = tid; i < kMaskWords; i += kThreads) {
@@ -1404,10 +1405,18 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     p.route = L.route;
     p.topk = L.topk;
     p.topp = L.topp;
+    // The split is decided for the whole call (a launch may cover one head group of it) and each
+    // launch splits its own units that fall among the call's last ones, so that a call run in
+    // head groups gives the same output as one launch.
     const long long units = static_cast<long long>(p.npairs) * L.BH;
-    const long long S = L.split_all ? std::min<long long>(units, std::max(L.split_cap, 0))
-                                    : split_units(units, 2 * sm_count[dev], L.split_cap);
-    p.split_first = static_cast<int>(units - S);
+    const long long call_units = L.call_units > 0 ? L.call_units : units;
+    const long long S_call = L.split_all ? std::min<long long>(call_units, std::max(L.split_cap, 0))
+                                         : split_units(call_units, 2 * sm_count[dev], L.split_cap);
+    const long long first_call = call_units - S_call;
+    const long long first_local = std::min(units, std::max(0LL, first_call - L.unit0));
+    const long long S = units - first_local;
+    p.split_first = static_cast<int>(first_local);
+    p.split_slot0 = static_cast<int>(L.unit0 + first_local - first_call);
     p.split_cnt = L.split_cnt;
     p.split_part = L.split_part;
     const long long grid = units + S;
