@@ -140,10 +140,14 @@ Pooled pooled_at(void *workspace, const Shape &full, int bh0, bool with_split = 
 // counters (the kernel also returns each counter it uses to zero).
 constexpr size_t kClearBytes = kSplitCntOffset + 4 * static_cast<size_t>(kSplitCap);
 
-// Pool K, V of the s.BH heads starting at k, v into `pw` (no argument checks).
-sol_status launch_pool(const void *k, const void *v, const Shape &s, const Pooled &pw, cudaStream_t stream)
+// Pool K, V of the s.BH heads starting at k, v into `pw` (no argument checks); with clear_header
+// the pool kernel also zeroes the workspace header's status words and split counters.
+sol_status launch_pool(const void *k, const void *v, const Shape &s, const Pooled &pw, cudaStream_t stream,
+                       bool clear_header)
 {
-    return launch_pool_kv(k, v, s.BH, s.N, s.Nk, s.d, pw.k32, pw.v32, pw.k16, pw.v16, stream) == cudaSuccess
+    int *clear = clear_header ? reinterpret_cast<int *>(pw.status) : nullptr;
+    return launch_pool_kv(k, v, s.BH, s.N, s.Nk, s.d, pw.k32, pw.v32, pw.k16, pw.v16, clear,
+                          static_cast<int>(kClearBytes / 4), stream) == cudaSuccess
                ? SOL_OK : SOL_ERR_CUDA;
 }
 
@@ -287,9 +291,8 @@ sol_status pool_fwd_unsplit(const void *q, const void *k, const void *v, int B, 
     if (st != SOL_OK) return st;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
     if (density && (reinterpret_cast<uintptr_t>(density) & 3u)) return SOL_ERR_ALIGNMENT;
-    if (cudaMemsetAsync(workspace, 0, kClearBytes, stream) != cudaSuccess) return SOL_ERR_CUDA;
     const Pooled pw = pooled_at(workspace, s, 0, false);
-    st = launch_pool(k, v, s, pw, stream);
+    st = launch_pool(k, v, s, pw, stream, true);
     if (st != SOL_OK) return st;
     return launch_fwd(q, k, v, s, pw, beta, nullptr, out, density, nullptr, nullptr, nullptr, 0,
                       kDefaultTimeoutNs, stream, RouteArg{});
@@ -318,8 +321,7 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
     if (st != SOL_OK) return st;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SOL_ERR_ALIGNMENT;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(workspace, 0, kClearBytes, cs) != cudaSuccess) return SOL_ERR_CUDA;
-    return launch_pool(k, v, s, pooled_at(workspace, s, 0), cs);
+    return launch_pool(k, v, s, pooled_at(workspace, s, 0), cs, true);
 }
 
 sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
@@ -470,7 +472,7 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
         gs.BH = h1 - h0;
         const Pooled pw = pooled_at(workspace, s, h0);
         int32_t *gd = d_density ? d_density + static_cast<size_t>(h0) * s.Nq : nullptr;
-        st = launch_pool(gk, gv, gs, pw, cs);
+        st = launch_pool(gk, gv, gs, pw, cs, false);   // the header was cleared once for the call
         if (st == SOL_OK)
             st = launch_fwd(gq, gk, gv, gs, pw, beta, nullptr, go, gd, nullptr, nullptr, nullptr, 0,
                             kDefaultTimeoutNs, cs, RouteArg{});

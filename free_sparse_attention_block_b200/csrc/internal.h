@@ -35,8 +35,11 @@ struct WorkspaceLayout {
 // with_split = false leaves out the split region (split_cap = 0: no tile pair is split).
 WorkspaceLayout workspace_layout(long long BH, long long Nk, int d, bool with_split = true);
 
+// clear (or null): block 0 of the pool also zeroes clear[0, clear_words), the workspace header's
+// status words and split counters, which the forward that follows in stream order reads.
 cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, int d, float *kbar32,
-                           float *vbar32, void *kbar16, void *vbar16, cudaStream_t stream);
+                           float *vbar32, void *kbar16, void *vbar16, int *clear, int clear_words,
+                           cudaStream_t stream);
 
 // Block-selection rule of the routing step.  The page's own rule is the threshold
 // mu + beta*sigma; top-k and top-p are the prior-art rules it compares against, run on the same

@@ -44,8 +44,11 @@ template <int D, int CPL>
 __global__ void __launch_bounds__(kPoolThreads) pool_kv_kernel(
     const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v, int BH, int N, int Nk,
     float *__restrict__ kbar32, float *__restrict__ vbar32, __nv_bfloat16 *__restrict__ kbar16,
-    __nv_bfloat16 *__restrict__ vbar16)
+    __nv_bfloat16 *__restrict__ vbar16, int *__restrict__ clear, int clear_words)
 {
+    if (blockIdx.x == 0 && clear != nullptr) {
+        for (int i = threadIdx.x; i < clear_words; i += kPoolThreads) clear[i] = 0;
+    }
     using Vec = typename RowVec<CPL>::T;
     constexpr int kLanes = D / CPL;                        // lanes per block = vectors per token row
     const long long grp = (static_cast<long long>(blockIdx.x) * kPoolThreads + threadIdx.x) / kLanes;
@@ -90,7 +93,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kv_kernel(
 }  // namespace
 
 cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, int d, float *kbar32,
-                           float *vbar32, void *kbar16, void *vbar16, cudaStream_t stream)
+                           float *vbar32, void *kbar16, void *vbar16, int *clear, int clear_words,
+                           cudaStream_t stream)
 {
     if (!head_dim_supported(d)) return cudaErrorInvalidValue;
     constexpr int kCpl = SOL_POOL_CPL;
@@ -100,7 +104,8 @@ cudaError_t launch_pool_kv(const void *k, const void *v, int BH, int N, int Nk, 
     auto kern = d == 64 ? pool_kv_kernel<64, kCpl> : pool_kv_kernel<128, kCpl>;
     kern<<<static_cast<unsigned>(blocks), kPoolThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), BH, N, Nk,
-        kbar32, vbar32, static_cast<__nv_bfloat16 *>(kbar16), static_cast<__nv_bfloat16 *>(vbar16));
+        kbar32, vbar32, static_cast<__nv_bfloat16 *>(kbar16), static_cast<__nv_bfloat16 *>(vbar16), clear,
+        clear_words);
     return cudaGetLastError();
 }
 
