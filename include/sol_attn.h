@@ -150,6 +150,8 @@ sol_status sol_attn_fwd_debug_route(const void *q, const void *k, const void *v,
  *               runs out and the call must return SOL_ERR_TIMEOUT with the context intact.
  *               bit 1: split every work unit the workspace has room for (up to 128 tile pairs)
  *               over two CTAs, whatever the wave shape (tests of the merge on small shapes).
+ *               bit 2: the first half of a split unit publishes its rows but not its final
+ *               count, so the other half's wait for them runs out (SOL_ERR_TIMEOUT).
  *   timeout_ms: limit for each device wait; <= 0 selects the production default (2000 ms).
  * Returns SOL_ERR_TIMEOUT if any device wait ran out, else the launch status. */
 sol_status sol_attn_fwd_debug(const void *q, const void *k, const void *v, int B, int H, int N,

@@ -25,3 +25,20 @@ def test_stalled_wait_reports_timeout_and_context_survives():
     assert sol.sol_attn_read_status(ws)[0] == 0
     g = gpu_run(q, k, v, 0.5)
     check_parity(q, k, v, 0.5, g, default_units(2, 8, None))
+
+
+def test_split_merge_wait_reports_timeout_and_context_survives():
+    """The second half of a split work unit waits (bounded) for the first half's rows; with the
+    first half's final count withheld (fault flag 4, every unit split by flag 2) that wait must
+    run out, report SOL_ERR_TIMEOUT and leave the context usable."""
+    N = 64 * 8
+    q, k, v = inputs.small_workload(N, BH=2, seed=6)
+    tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+    ws = torch.zeros(sol.sol_attn_workspace_bytes(1, 2, N, 128), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(tq)
+    sol.sol_attn_pool(tk, tv, ws)
+    st = sol.sol_attn_fwd_debug(tq, tk, tv, 0.5, ws, out, fault_flags=2 | 4, timeout_ms=50)
+    assert sol.STATUS[st] == "SOL_ERR_TIMEOUT"
+    assert sol.sol_attn_read_status(ws)[0] == 0
+    g = gpu_run(q, k, v, 0.5)
+    check_parity(q, k, v, 0.5, g, default_units(2, 8, None))
