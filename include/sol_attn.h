@@ -32,8 +32,10 @@
  *   - Device-side failures (a pipeline wait that ran out of time) are recorded in a status word
  *     inside the workspace; sol_attn_read_status() synchronises the stream and returns it.
  *   - The library keeps no state between calls apart from per-device one-time set-up (kernel
- *     attributes, the driver entry point for tensor-map encoding, and the two copy streams and
- *     the events sol_attn_fwd_host pipelines its copies with); it is thread-safe.
+ *     attributes, the SM count that sizes the split of the last wave of CTAs, the driver entry
+ *     point for tensor-map encoding, and the two copy streams and the events sol_attn_fwd_host
+ *     pipelines its copies with); it is thread-safe.  Calls that share a workspace must not
+ *     overlap on the GPU.
  */
 #ifndef SOL_ATTN_H
 #define SOL_ATTN_H
