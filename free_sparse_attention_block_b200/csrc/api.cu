@@ -382,7 +382,8 @@ sol_status sol_attn_fwd_debug_route(const void *q, const void *k, const void *v,
 
 sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream)
 {
-    if (!workspace) return SOL_ERR_INVALID_ARG;
+    // NULL: the status words of sol_attn_fwd_noalloc's built-in scratch on the current device
+    if (!workspace && noalloc_scratch(&workspace) != cudaSuccess) return SOL_ERR_CUDA;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(cs) != cudaSuccess) return SOL_ERR_CUDA;
     DeviceStatus h{};

@@ -64,12 +64,17 @@ struct FwdLaunch {
     int topk;       // kRouteTopK: blocks kept per query tile
     float topp;     // kRouteTopP: probability mass covered per query tile
     int split_cap;  // tile pairs the workspace can split (0: none)
-    int *split_cnt;       // [split_cap] arrival counters, zero between calls
+    int *split_cnt;       // [split_cap] arrival counters (launch tag << 2 | count); a merging CTA
+                          // returns its counter to 0, and a stale tag counts as 0
     float *split_part;    // [split_cap][2][128][d + 4] partial rows
     bool split_all;       // split every tile pair up to split_cap (test entry point)
     long long call_units; // tile pairs of the whole call this launch is part of (its head groups)
     long long unit0;      // the call's index of this launch's first tile pair
 };
 cudaError_t launch_sol_fwd(const FwdLaunch &L, cudaStream_t stream);
+
+// Device address of sol_attn_fwd_noalloc's built-in scratch on the current device (looked up once
+// per device and cached; a failed lookup is not cached, so the next call retries).
+cudaError_t noalloc_scratch(void **addr);
 
 }  // namespace sol

@@ -6,9 +6,10 @@
 //
 // The array is a host-side stand-in for a device symbol: host code must never pass its name to a
 // kernel.  Its device address is obtained once per device with cudaGetSymbolAddress, with that
-// device current, and cached.
+// device current, and cached once the lookup succeeds.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -19,9 +20,8 @@ namespace {
 __device__ __align__(256) unsigned char g_noalloc_scratch[SOL_ATTN_NOALLOC_MAX_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void *g_addr[kMaxDevices];
-cudaError_t g_err[kMaxDevices];
+std::mutex g_mu;
+std::atomic<void *> g_addr[kMaxDevices];
 
 sol_status shape_error(int B, int H, int N, int d)
 {
@@ -35,7 +35,32 @@ sol_status shape_error(int B, int H, int N, int d)
 namespace sol {
 sol_status pool_fwd_unsplit(const void *q, const void *k, const void *v, int B, int H, int N, int d,
                             float beta, void *workspace, void *out, int32_t *density, cudaStream_t stream);
+
+cudaError_t noalloc_scratch(void **addr)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    void *a = g_addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        // Only a successful lookup is cached: one made during a stream capture, or after a
+        // transient error, is retried by the next call.
+        std::lock_guard<std::mutex> lock(g_mu);
+        a = g_addr[dev].load(std::memory_order_relaxed);
+        if (!a) {
+            e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+            if (e != cudaSuccess || !a) {
+                cudaGetLastError();   // do not leave the error for a later launch check to report
+                return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+            }
+            g_addr[dev].store(a, std::memory_order_release);
+        }
+    }
+    *addr = a;
+    return cudaSuccess;
 }
+}  // namespace sol
 
 extern "C" sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const void *v, int B,
                                            int H, int N, int d, float beta, void *out,
@@ -47,15 +72,11 @@ extern "C" sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const v
     const size_t need = sol::workspace_layout(BH, Nk, d, false).total;
     if (need > SOL_ATTN_NOALLOC_MAX_BYTES) return SOL_ERR_SCRATCH_LIMIT;
 
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SOL_ERR_CUDA;
-    std::call_once(g_once[dev], [dev] {
-        g_err[dev] = cudaGetSymbolAddress(&g_addr[dev], g_noalloc_scratch);
-    });
-    if (g_err[dev] != cudaSuccess || g_addr[dev] == nullptr) return SOL_ERR_CUDA;
+    void *scratch = nullptr;
+    if (sol::noalloc_scratch(&scratch) != cudaSuccess) return SOL_ERR_CUDA;
 
     // The pool clears the status words and overwrites every pooled row the forward reads, so
     // nothing left in the array by an earlier call is used.  The scratch has no split region.
-    return sol::pool_fwd_unsplit(q, k, v, B, H, N, d, beta, g_addr[dev], out, density_out,
+    return sol::pool_fwd_unsplit(q, k, v, B, H, N, d, beta, scratch, out, density_out,
                                  static_cast<cudaStream_t>(stream));
 }

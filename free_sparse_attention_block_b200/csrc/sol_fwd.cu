@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstddef>
 #include <mutex>
@@ -169,7 +170,8 @@ struct Params {
     float topp;              // probability mass to cover per query tile (top-p)
     int split_first;         // units from this one on run as two CTAs each (the unit count: none)
     int split_slot0;         // the call's split slot of unit split_first (head groups of one call)
-    int *split_cnt;          // arrival counter per split unit, zero between calls
+    int *split_cnt;          // arrival counter per split unit: launch tag << 2 | count
+    int split_gen;           // this launch's tag (nonzero); another tag in a counter reads as 0
     float *split_part;       // [split unit][half][128 rows][D + 4] partial rows
 };
 
@@ -527,6 +529,21 @@ __device__ __forceinline__ bool softmax_item(uint32_t tmem, Misc &m, const Param
     return true;
 }
 
+// Arrival of one half of a split unit on its counter, which holds (launch tag << 2) | count.  A
+// counter whose tag is not this launch's counts as 0: a launch that gave up part way (a wait ran
+// out) may leave its counters at 1 or 2, and a later launch on the same workspace must not read
+// them as arrivals.  Returns the count before this arrival.
+__device__ __forceinline__ int split_arrive(int *cnt, int gen)
+{
+    int old = *reinterpret_cast<volatile int *>(cnt);
+    for (;;) {
+        const int c = (old >> 2) == gen ? (old & 3) : 0;
+        const int prev = atomicCAS(cnt, old, (gen << 2) | (c + 1));
+        if (prev == old) return c;
+        old = prev;
+    }
+}
+
 // Epilogue of a unit split over two CTAs; softmax threads, one per row (TMEM lane).  Each half
 // counts its arrival on the unit's counter.  The first to arrive writes its rows' unnormalised
 // output O (relative to 2^m), running max m (log2 domain) and sum l to its partial slot and counts
@@ -557,7 +574,7 @@ __device__ __forceinline__ void split_epilogue(uint32_t tmem, Misc &m, const Par
     // Arrival first: the first half to arrive publishes its rows and counts again (the counter
     // reaches 3 once both halves have arrived and the rows are out); the second merges and never
     // writes its own partial rows.
-    if (row == 0) m.split_old = atomicAdd(cnt, 1);
+    if (row == 0) m.split_old = split_arrive(cnt, p.split_gen);
     asm volatile("bar.sync 1, %0;" ::"r"(kSoftmaxThreads) : "memory");
     if (m.split_old == 0) {
         float *mine = p.split_part + (static_cast<size_t>(2 * slot + half) * kBM + row) * kRow;
@@ -581,7 +598,8 @@ __device__ __forceinline__ void split_epilogue(uint32_t tmem, Misc &m, const Par
         mine[D + 1] = l;
         __threadfence();                                           // the rows are visible ...
         asm volatile("bar.sync 1, %0;" ::"r"(kSoftmaxThreads) : "memory");
-        // ... before this count (debug fault flag 4 withholds it, so the other half's wait runs out)
+        // ... before this count (debug fault flag 4 withholds it, so the other half's wait runs
+        // out); the counter already carries this launch's tag
         if (row == 0 && !(p.fault_flags & 4)) atomicAdd(cnt, 1);
         return;
     }
@@ -589,17 +607,18 @@ __device__ __forceinline__ void split_epilogue(uint32_t tmem, Misc &m, const Par
     // arrived, so it is running and its publication ends.
     if (row == 0) {
         const uint64_t t0 = globaltimer_ns();
+        const int done = (p.split_gen << 2) | 3;
         int seen;
         for (;;) {
             asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(cnt) : "memory");
-            if (seen >= 3) break;
+            if (seen == done) break;
             if (globaltimer_ns() - t0 > p.timeout_ns) {
                 if (atomicCAS(&p.status->code, 0, 5) == 0) atomicExch(&p.status->where, kSiteMerge);
                 break;
             }
             __nanosleep(256);
         }
-        m.split_old = seen >= 3 ? 1 : -1;
+        m.split_old = seen == done ? 1 : -1;
     }
     asm volatile("bar.sync 1, %0;" ::"r"(kSoftmaxThreads) : "memory");
     if (m.split_old < 0) return;
@@ -1420,6 +1439,9 @@ cudaError_t launch_d(const FwdLaunch &L, cudaStream_t stream)
     p.split_slot0 = static_cast<int>(L.unit0 + first_local - first_call);
     p.split_cnt = L.split_cnt;
     p.split_part = L.split_part;
+    // a fresh tag per launch, 1 .. 2^29 - 1 (tag << 2 | count stays a positive int)
+    static std::atomic<unsigned> launch_tag{0};
+    p.split_gen = static_cast<int>(launch_tag.fetch_add(1u, std::memory_order_relaxed) % 0x1FFFFFFFu) + 1;
     const long long grid = units + S;
     if (units <= 0 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     sol_fwd_kernel<D, kRank><<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(

@@ -74,8 +74,12 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 to bfloat16 (nearest, ties to even); returns uint16 bit patterns."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     u = x.view(np.uint32)
-    bias = ((u >> 16) & 1) + np.uint32(0x7FFF)
-    out = ((u + bias) >> 16).astype(np.uint16)
+    r = np.right_shift(u, 16)          # in place from here on: one uint32 temporary
+    r &= np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= np.uint32(16)
+    out = r.astype(np.uint16)
     nan = np.isnan(x)
     if nan.any():
         out[nan] = 0x7FC0
@@ -89,8 +93,10 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 def _field(rng: np.random.Generator, grid, d: int, f_max: float) -> np.ndarray:
     """Sum of 4 random sinusoids per channel over the (T, H, W) grid -> float32 [N, d].
 
-    The phase is separable, angle = a(t) + b(y) + c(x) + phi, so each term is evaluated as
-    Im(e^{i a} e^{i b} e^{i (c + phi)}) with the small per-axis exponentials broadcast over the grid.
+    The phase is separable, angle = a(t) + b(y) + (c(x) + phi), so with A = a + b and
+    C = c + phi each term is sin(A) cos(C) + cos(A) sin(C): per channel, the field over
+    ((t, y), x) is a product of a [T*H, 8] and an [8, W] matrix (4 terms x 2 products), evaluated
+    in float64 as one batched matrix product over the channels.
     """
     T, Hg, Wg = grid
     f = rng.uniform(0.0, f_max, size=(d, 4, 3))
@@ -98,15 +104,14 @@ def _field(rng: np.random.Generator, grid, d: int, f_max: float) -> np.ndarray:
     t = np.arange(T, dtype=np.float64) / T
     y = np.arange(Hg, dtype=np.float64) / Hg
     x = np.arange(Wg, dtype=np.float64) / Wg
-    out = np.zeros((T, Hg, Wg, d), dtype=np.float64)
-    for s in range(4):
-        ea = np.exp(2j * math.pi * f[:, s, 0][None, :] * t[:, None])                  # [T, d]
-        eb = np.exp(2j * math.pi * f[:, s, 1][None, :] * y[:, None])                  # [H, d]
-        ec = np.exp(1j * (2.0 * math.pi * f[:, s, 2][None, :] * x[:, None] + phi[:, s][None, :]))  # [W, d]
-        eab = ea[:, None, :] * eb[None, :, :]                                          # [T, H, d]
-        out += eab.real[:, :, None, :] * ec.imag[None, None, :, :]
-        out += eab.imag[:, :, None, :] * ec.real[None, None, :, :]
-    return out.reshape(T * Hg * Wg, d).astype(np.float32)
+    ang_a = 2.0 * math.pi * (f[None, None, :, :, 0] * t[:, None, None, None] +
+                             f[None, None, :, :, 1] * y[None, :, None, None])         # [T, H, d, 4]
+    ang_c = 2.0 * math.pi * f[None, :, :, 2] * x[:, None, None] + phi[None, :, :]   # [W, d, 4]
+    left = np.concatenate([np.sin(ang_a), np.cos(ang_a)], axis=3).reshape(T * Hg, d, 8)
+    right = np.concatenate([np.cos(ang_c), np.sin(ang_c)], axis=2)                     # [W, d, 8]
+    prod = np.matmul(np.ascontiguousarray(left.transpose(1, 0, 2)),
+                     np.ascontiguousarray(right.transpose(1, 2, 0)))                   # [d, T*H, W]
+    return np.ascontiguousarray(prod.transpose(1, 2, 0), dtype=np.float32).reshape(T * Hg * Wg, d)
 
 
 def gen_head(seed: int, b: int, h: int, grid, d: int = HEAD_DIM, f_max: float = 1.5,
@@ -120,21 +125,23 @@ def gen_head(seed: int, b: int, h: int, grid, d: int = HEAD_DIM, f_max: float = 
     n = F.shape[0] if n_tokens is None else n_tokens
     assert n <= F.shape[0]
     F = F[:n]
-    q = 0.5 * F + rng.standard_normal((n, d), dtype=np.float32)
-    k = 0.5 * F + rng.standard_normal((n, d), dtype=np.float32)
-    v = rng.standard_normal((n, d), dtype=np.float32)
-    return f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(v)
-
-
-def _gen_head_star(args):
-    return gen_head(*args)
+    F *= np.float32(0.5)                  # exact; 0.5*F + noise below, in float32
+    out = []
+    for with_field in (True, True, False):   # q, k (field + noise), then v (noise)
+        x = rng.standard_normal((n, d), dtype=np.float32)
+        if with_field:
+            x += F
+        out.append(f32_to_bf16_bits(x))
+    return tuple(out)
 
 
 def gen_workload(wl: Workload, heads=None, processes: int | None = None, n_tokens: int | None = None):
     """All heads of a workload: q, k, v uint16 [B, H, N, d].
 
     ``heads`` restricts generation to a list of (b, h) pairs (others are left zero).
-    Large workloads are generated in a spawn-started process pool (safe after CUDA init).
+    Heads are generated by a pool of threads (numpy releases the GIL in the random draws, the
+    matrix products and the element-wise passes), each writing its own slices of the outputs;
+    ``processes`` caps the thread count (default: the usable cores, at most 32).
     """
     n = wl.N if n_tokens is None else n_tokens
     shape = (wl.B, wl.H, n, wl.d)
@@ -142,17 +149,22 @@ def gen_workload(wl: Workload, heads=None, processes: int | None = None, n_token
     k = np.zeros(shape, np.uint16)
     v = np.zeros(shape, np.uint16)
     todo = [(b, h) for b in range(wl.B) for h in range(wl.H)] if heads is None else list(heads)
-    args = [(wl.seed, b, h, wl.grid, wl.d, wl.f_max, n) for (b, h) in todo]
+
+    def one(bh):
+        b, h = bh
+        q[b, h], k[b, h], v[b, h] = gen_head(wl.seed, b, h, wl.grid, wl.d, wl.f_max, n)
+
     if processes is None:
-        processes = min(len(todo), os.cpu_count() or 1, 16) if n * len(todo) > 4_000_000 else 1
-    if processes > 1:
-        import multiprocessing as mp
-        with mp.get_context("spawn").Pool(processes) as pool:
-            results = pool.map(_gen_head_star, args, chunksize=1)
+        processes = min(len(todo), len(os.sched_getaffinity(0)), 32) if n * len(todo) > 4_000_000 else 1
+    if processes > 1 and len(todo) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"), ThreadPoolExecutor(processes) as ex:
+            list(ex.map(one, todo))   # one BLAS thread per head: the heads are the parallelism
     else:
-        results = [_gen_head_star(a) for a in args]
-    for (b, h), (qh, kh, vh) in zip(todo, results):
-        q[b, h], k[b, h], v[b, h] = qh, kh, vh
+        for bh in todo:
+            one(bh)
     return q, k, v
 
 

@@ -162,8 +162,12 @@ sol_status sol_attn_fwd_debug(const void *q, const void *k, const void *v, int B
                               float *stats_out, int fault_flags, int timeout_ms, void *stream);
 
 /* Synchronise `stream`, read the device status words in the workspace header and clear them.
- * Returns SOL_OK, SOL_ERR_TIMEOUT (a device wait gave up) or SOL_ERR_CUDA.  If where_out is not
- * NULL it receives an internal code naming the wait that gave up (0 if none). */
+ * workspace NULL reads the status words of sol_attn_fwd_noalloc's built-in scratch on the current
+ * device instead.  Returns SOL_OK, SOL_ERR_TIMEOUT (a device wait gave up) or SOL_ERR_CUDA.  If
+ * where_out is not NULL it receives an internal code naming the wait that gave up (0 if none).
+ * A call that gave up leaves no state that misleads a later call on the same workspace, whether or
+ * not its status was read: the counters of split tile pairs carry a tag of the launch that wrote
+ * them, and another launch's tag counts as zero. */
 sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream);
 
 /* One end-to-end call on host buffers: copies q, k, v from (preferably pinned) host memory into
@@ -200,13 +204,13 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
  *     CTAs may run less full than sol_attn_fwd's.
  *   - The first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any stream
- *     capture.
+ *     capture.  A lookup that fails returns SOL_ERR_CUDA and is retried by the next call.
  *   - Every call on a device shares the one array and leaves its contents behind; each call
  *     clears the status words and rewrites all pooled rows it reads before use.  Calls whose
  *     execution overlaps on the GPU (different streams, or graphs launched concurrently) race on
  *     the array: serialise them.
- *   - Device-side wait timeouts are recorded in the scratch status words, which the caller cannot
- *     address; use sol_attn_fwd with an own workspace to read them.
+ *   - Device-side wait timeouts are recorded in the scratch status words; sol_attn_read_status
+ *     with a NULL workspace synchronises the stream and reads (and clears) them.
  * Other arguments, errors and asynchrony as for sol_attn_fwd. */
 sol_status sol_attn_fwd_noalloc(const void *q, const void *k, const void *v, int B, int H, int N,
                                 int d, float beta, void *out, int32_t *density_out, void *stream);

@@ -127,11 +127,3 @@ def forward(q, k, v, beta: float, units=None, mask_override=None):
     r["kbar"], r["vbar"] = kbar, vbar
     return r
 
-
-def gather_rows(out_units, units, N: int, Nq: int):
-    """Flatten [U, 64, d] tile outputs into ((bh, token) index arrays, rows) for tokens < N."""
-    bh = units // Nq
-    i = units % Nq
-    tok = i[:, None] * TILE + np.arange(TILE)[None, :]
-    valid = tok < N
-    return bh[:, None].repeat(TILE, 1)[valid], tok[valid], out_units[valid]

@@ -1,7 +1,8 @@
 """sol_attn_fwd_sharded through a one-rank NCCL group on one GPU: the sharded entry point (head
-range, CUDA forward of the rank's heads, NCCL all-gather of outputs and densities) must return
-exactly what the single-GPU forward returns.  The multi-rank gather itself is covered on CPU with
-gloo (tests/test_sharded.py)."""
+range, CUDA forward of the rank's heads, NCCL all-gather of outputs and densities) is checked
+against the oracle on every tile (with the GPU's own masks from the debug outputs for near ties)
+and must return exactly what the single-GPU forward returns.  The multi-rank gather itself is
+covered on CPU with gloo (tests/test_sharded.py)."""
 import datetime
 import os
 import socket
@@ -14,11 +15,12 @@ import torch.distributed as dist
 import free_sparse_attention_block_b200 as sol
 from free_sparse_attention_block_b200 import inputs
 from free_sparse_attention_block_b200.sharded import sol_attn_fwd_sharded
+from parity import check_parity, default_units, gpu_run
 
 pytestmark = pytest.mark.gpu
 
 
-def test_one_rank_nccl_group_matches_the_single_gpu_forward():
+def test_one_rank_nccl_group_against_the_oracle():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
@@ -35,6 +37,9 @@ def test_one_rank_nccl_group_matches_the_single_gpu_forward():
         torch.cuda.synchronize()
         assert torch.equal(got_out.view(torch.int16), want_out.view(torch.int16))
         assert torch.equal(got_dens, want_dens)
+        ref = gpu_run(q, k, v, 0.7)           # the GPU's masks and statistics (debug outputs)
+        g = dict(ref, out=got_out.float().cpu().numpy(), density=got_dens.cpu().numpy())
+        check_parity(q, k, v, 0.7, g, default_units(H, (N + 63) // 64, None))
         with pytest.raises(ValueError):
             sol_attn_fwd_sharded(tq[:, :4], tk[:, :4], tv[:, :4], 0.7, H)   # not this rank's heads
     finally:

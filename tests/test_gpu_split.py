@@ -11,7 +11,7 @@ import torch
 
 import free_sparse_attention_block_b200 as sol
 from free_sparse_attention_block_b200 import inputs
-from parity import check_parity, default_units, to_dev
+from parity import check_parity, check_rule_parity, default_units, gpu_run_rule, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -80,3 +80,15 @@ def test_production_split_of_the_last_wave_on_mid():
     q, k, v = inputs.gen_workload(wl, heads=[(0, 11)])
     g = split_run(q, k, v, 0.5, flags=0)
     check_parity(q, k, v, 0.5, g, np.arange(11 * wl.nq, 12 * wl.nq, dtype=np.int64))
+
+
+@pytest.mark.parametrize("rule,param", [("topk", 62), ("topp", 0.5)])
+def test_production_split_of_the_last_wave_rank_rules(rule, param):
+    """The rank rules' kernel splits the same last 84 units of the 12-head, 16384-token call
+    (after its radix selection); the last head's tiles against the oracle's selection and
+    outputs."""
+    wl = inputs.WORKLOADS["mid"]
+    q, k, v = inputs.gen_workload(wl, heads=[(0, 11)])
+    units = np.arange(11 * wl.nq, 12 * wl.nq, dtype=np.int64)
+    g = gpu_run_rule(q, k, v, rule, param, units=units)
+    check_rule_parity(q, k, v, rule, param, g)

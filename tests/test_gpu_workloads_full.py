@@ -1,7 +1,10 @@
 """Full-size workloads (Wan2.1-14B-shaped, HunyuanVideo-shaped, long-video stress) in the launch
-configuration the benchmark times (sol_attn_pool + sol_attn_fwd over all heads), checked against
-the oracle on sampled query tiles: per head the first, second, second-to-last and last tile (the
-last one partial for Wan and Hunyuan) plus random ones."""
+configuration the benchmark times (sol_attn_pool + sol_attn_fwd over all heads), over each
+workload's whole beta sweep, checked against the oracle on sampled query tiles: per head the
+first, second, second-to-last and last tile (the last one partial for Wan and Hunyuan) plus random
+ones, on four heads.  One case runs the Wan2.1 shape with 64-channel heads."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -10,13 +13,25 @@ from parity import check_parity, default_units, gpu_run
 
 pytestmark = pytest.mark.gpu
 
-CASES = [("wan", 0.5), ("wan", 2.0), ("hunyuan", 1.0), ("long", 2.0)]
+CASES = ([("wan", 128, b) for b in (0.5, 1.0, 1.5, 2.0)] + [("wan", 64, 0.5)] +
+         [("hunyuan", 128, b) for b in (0.5, 1.0, 1.5, 2.0, 2.5)] +
+         [("long", 128, b) for b in (1.5, 2.0, 2.5)])
+
+_last = {}
 
 
-@pytest.mark.parametrize("name,beta", CASES)
-def test_full_size_sampled(name, beta):
-    wl = inputs.WORKLOADS[name]
-    q, k, v = inputs.gen_workload(wl)
+def workload_inputs(name, d):
+    """Inputs of one workload, kept while consecutive cases use it (one workload at a time)."""
+    if (name, d) not in _last:
+        _last.clear()
+        wl = dataclasses.replace(inputs.WORKLOADS[name], d=d)
+        _last[(name, d)] = (wl, inputs.gen_workload(wl))
+    return _last[(name, d)]
+
+
+@pytest.mark.parametrize("name,d,beta", CASES)
+def test_full_size_sampled(name, d, beta):
+    wl, (q, k, v) = workload_inputs(name, d)
     BH, Nq = wl.B * wl.H, wl.nq
     rng = np.random.default_rng(wl.seed)
     heads = sorted({0, BH - 1, *rng.integers(0, BH, size=2).tolist()})
@@ -25,4 +40,8 @@ def test_full_size_sampled(name, beta):
     g = gpu_run(q, k, v, beta, units=units, with_proxy=True)
     rep = {}
     check_parity(q, k, v, beta, g, units, report=rep)
-    print(f"{name} beta={beta}: {rep}")
+    print(f"{name} d={d} beta={beta}: {rep}")
+
+
+def teardown_module():
+    _last.clear()
