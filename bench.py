@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the Sol-Attn forward (pool + fused routing/attention) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid] [--beta 0.5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--beta 1.5]
     python bench.py --impl reference ...      # the CPU oracle on the host cores
 
 One step = sol_attn_pool + sol_attn_fwd over one batch of the seeded synthetic workload (the
@@ -37,10 +37,11 @@ from free_sparse_attention_block_b200 import inputs  # noqa: E402
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
-# DRAM bytes (read + write) per launch of the fused kernel from one ncu capture, keyed by
-# (workload, head dim, beta), valid only for the kernel source whose sha256 prefix is given.
+# DRAM bytes (read + write) per head of one launch of the fused kernel, from one ncu capture of a
+# launch over the workload's first heads (heads are independent, so traffic scales with them),
+# keyed by (workload, head dim, beta); valid only for the kernel source whose sha256 prefix is given.
 NCU_TRAFFIC = {
-    ("mid", 128, 0.5): {"bytes": 154706432 + 33871872, "kernel": "a5565cff4574a267"},
+    ("mid", 128, 0.5): {"bytes_per_head": (154706432 + 33871872) / 12, "kernel": "a5565cff4574a267"},
 }
 
 
@@ -179,6 +180,32 @@ def flop_counts(mask: np.ndarray, N: int, d: int = 128):
     density_tokens = kept / (4.0 * d * BH * float(N) ** 2)
     return dict(kept=kept, corr=corr, executed=executed, density=float(mask.mean()),
                 density_tokens=density_tokens)
+
+
+def mask_flop_counts(mask, N: int, d: int = 128):
+    """flop_counts computed with torch on the mask's own device (the full-size masks stay on the
+    GPU): mask is a uint8 tensor [BH, Nq, Nk].  Same definitions and results as flop_counts."""
+    import torch
+    BH, Nq, Nk = mask.shape
+    n_last = N - 64 * (Nk - 1)
+    n = torch.full((Nq,), 64, dtype=torch.int64, device=mask.device)
+    n[-1] = n_last
+    cnt = mask.sum(-1, dtype=torch.int64)                                   # kept blocks per tile
+    row = 64 * cnt - (64 - n_last) * mask[..., -1].to(torch.int64)       # sum_j kept n_j per tile
+    kept = 4.0 * d * float((row * n).sum())
+    corr = 4.0 * d * float(((Nk - cnt) * n).sum())
+    m = mask.bool()
+    if Nq % 2:
+        m = torch.cat([m, torch.ones((BH, 1, Nk), dtype=torch.bool, device=mask.device)], dim=1)
+    a, b = m[:, 0::2], m[:, 1::2]
+    union = int((a | b).sum())
+    nchunks = (Nk + 63) // 64
+    both = torch.cat([a & b, torch.ones((BH, a.shape[1], nchunks * 64 - Nk), dtype=torch.bool,
+                                        device=mask.device)], dim=2)
+    corr_chunks = int((~both.view(BH, a.shape[1], nchunks, 64).all(-1)).sum())
+    executed = 4.0 * d * 128 * 64 * float(union + corr_chunks)
+    return dict(kept=kept, corr=corr, executed=executed, density=float(cnt.sum()) / (BH * Nq * Nk),
+                density_tokens=kept / (4.0 * d * BH * float(N) ** 2))
 
 
 def density_spread(dens: np.ndarray, Nk: int) -> dict:
@@ -335,6 +362,75 @@ def config_of(wl, args):
                             else f"replicas x{args.gpus}")}
 
 
+def timed_fwd(fn, flush, stream, steps: int) -> float:
+    """Mean device time (ms) of ``fn`` over ``steps`` calls, L2 flushed before each."""
+    import torch
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in ts]))
+
+
+def beta_point(sol, wl, tq, tk, tv, ws, out, dens, beta, flush, stream, steps, dense):
+    """One (workload, beta) point: the kernel's own mask for the flop count, then the timed fwd."""
+    import torch
+    B, H, N, d = tq.shape
+    Nq = wl.nq
+    m = torch.empty((B * H, Nq, Nq), dtype=torch.uint8, device=tq.device)
+    st = sol.sol_attn_fwd_debug(tq, tk, tv, beta, ws, out, dens, None, m, None)
+    if st != 0:
+        raise RuntimeError(f"debug forward failed: {sol.STATUS.get(st)}")
+    fc = mask_flop_counts(m, N, d)
+    del m
+    ms = timed_fwd(lambda: sol.sol_attn_fwd(tq, tk, tv, beta, ws, out, dens), flush, stream, steps)
+    return {"beta": beta, "density": round(fc["density"], 4),
+            "density_tokens": round(fc["density_tokens"], 4), "fwd_ms": round(ms, 4),
+            "dense_equiv_tflops": round(dense / (ms * 1e-3) / 1e12, 1),
+            "computed_tile_frac": round(fc["kept"] / (ms * 1e-3) / 1e12 / PEAK_BF16, 4),
+            "computed_tile_frac_sustained": round(fc["kept"] / (ms * 1e-3) / 1e12 / PEAK_BF16_SUST, 4),
+            "roofline_frac": round((fc["kept"] + fc["corr"]) / (ms * 1e-3) / 1e12 / PEAK_BF16, 4)}
+
+
+def dense_regime(sol, dev, flush, stream, steps: int, d: int):
+    """The Wan2.1- and HunyuanVideo-shaped workloads at beta = 0.25 and 0 (block density 0.3 and
+    0.4, the regime of the tensor-peak target), each point timed (fwd only, L2 flushed) with its
+    own clock record."""
+    import torch
+    res = []
+    for name in ("wan", "hunyuan"):
+        wl = dataclasses.replace(inputs.WORKLOADS[name], d=d)
+        q, k, v = inputs.gen_workload(wl)
+        to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+        del q, k, v
+        B, H, N, _ = tq.shape
+        ws = torch.zeros(sol.sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+        out = torch.empty_like(tq)
+        dens = torch.empty((B, H, wl.nq), dtype=torch.int32, device=dev)
+        sol.sol_attn_pool(tk, tv, ws)
+        for beta in (0.25, 0.0):
+            for _ in range(2):
+                sol.sol_attn_fwd(tq, tk, tv, beta, ws, out, dens)
+            sampler = ClockSampler(dev)
+            with sampler:
+                pt = beta_point(sol, wl, tq, tk, tv, ws, out, dens, beta, flush, stream, steps,
+                                wl.dense_flops())
+            clk = sampler.summary()
+            res.append({"workload": name, **pt, "clocks": {k2: clk.get(k2) for k2 in ("sm_mhz", "reasons")}})
+        st, where = sol.sol_attn_read_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {sol.STATUS.get(st)} at wait site {where}")
+        del tq, tk, tv, ws, out, dens
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -346,13 +442,14 @@ def run_ours(args, wl):
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     sol.load_library()
 
     shard = args.shard == "heads"
+    t_gen = time.perf_counter()
     if shard:
         # this rank's contiguous head range; the outputs are all-gathered inside every step
         from free_sparse_attention_block_b200.sharded import gather_heads, head_range
@@ -361,12 +458,18 @@ def run_ours(args, wl):
             raise SystemExit(f"--shard heads: {wl.H} heads over {world} ranks leaves rank {rank} idle")
         q, k, v = inputs.gen_workload(wl, heads=[(b, h) for b in range(wl.B) for h in range(h0, h1)])
         q, k, v = (np.ascontiguousarray(x[:, h0:h1]) for x in (q, k, v))
+        hq, hk, hv = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v))
     else:
-        q, k, v = inputs.gen_workload(wl)
+        # generated straight into pinned host buffers: the end-to-end leg uploads from them
+        shape = (wl.B, wl.H, wl.N, wl.d)
+        hq, hk, hv = (torch.empty(shape, dtype=torch.int16, pin_memory=True) for _ in range(3))
+        q, k, v = (t.numpy().view(np.uint16) for t in (hq, hk, hv))
+        inputs.gen_workload(wl, out=(q, k, v))
+        hq, hk, hv = (t.view(torch.bfloat16) for t in (hq, hk, hv))
+    gen_s = time.perf_counter() - t_gen
     B, H, N, d = q.shape
     Nq = wl.nq
-    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
-    tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+    tq, tk, tv = (t.to(dev) for t in (hq, hk, hv))
     ws = torch.zeros(sol.sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
     out = torch.empty_like(tq)
     dens = torch.empty((B, H, Nq), dtype=torch.int32, device=dev)
@@ -375,11 +478,11 @@ def run_ours(args, wl):
 
     # mask once (outside timing) for the exact algorithmic flop count
     sol.sol_attn_pool(tk, tv, ws)
-    mask = torch.empty((B, H, Nq, Nq), dtype=torch.uint8, device=dev)
+    mask = torch.empty((B * H, Nq, Nq), dtype=torch.uint8, device=dev)
     st = sol.sol_attn_fwd_debug(tq, tk, tv, args.beta, ws, out, dens, None, mask, None)
     if st != 0:
         raise RuntimeError(f"debug forward failed: {sol.STATUS.get(st)}")
-    fc = flop_counts(mask.cpu().numpy().reshape(B * H, Nq, Nq), N, d)
+    fc = mask_flop_counts(mask, N, d)
     del mask
 
     def step(ev=None):
@@ -434,11 +537,8 @@ def run_ours(args, wl):
     value = dense / (t_max * 1e-3) / 1e12 if shard else replica_throughput(dense, world, t_max)
 
     # ---- e2e through the C ABI on pinned host buffers (copies inside the timed region)
-    hq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hk = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hv = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hout = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
-    hdens = torch.empty((B, H, Nq), dtype=torch.int32).pin_memory()
+    hout = torch.empty(hq.shape, dtype=torch.bfloat16, pin_memory=True)
+    hdens = torch.empty((B, H, Nq), dtype=torch.int32, pin_memory=True)
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
         sol.sol_attn_fwd_host(hq, hk, hv, args.beta, tq, tk, tv, ws, out, hout, dens, hdens)
@@ -451,37 +551,22 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     e2e_value = dense / (e2e_ms * 1e-3) / 1e12 if shard else replica_throughput(dense, world, e2e_ms)
-    assert torch.isfinite(hout.float()).all()
+    assert bool(torch.isfinite(hout[0, 0].float()).all()) and bool(torch.isfinite(hout[-1, -1].float()).all())
     h2d = 3 * B * H * N * d * 2
     d2h = B * H * N * d * 2 + B * H * Nq * 4
+    del hout
 
     # ---- beta sweep (fwd only, same inputs), for the record
     sweep = []
     if args.sweep:
         # the workload's beta sweep, plus 0.25 and 0.0 so that densities of 0.3 and above are covered
         for beta in sorted(set(wl.betas) | {0.0, 0.25}):
-            m2 = torch.empty((B, H, Nq, Nq), dtype=torch.uint8, device=dev)
-            sol.sol_attn_fwd_debug(tq, tk, tv, beta, ws, out, dens, None, m2, None)
-            fc2 = flop_counts(m2.cpu().numpy().reshape(B * H, Nq, Nq), N, d)
-            del m2
-            ts = []
-            for _ in range(max(3, args.steps // 2)):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                sol.sol_attn_fwd(tq, tk, tv, beta, ws, out, dens)
-                b.record(stream)
-                ts.append((a, b))
-            torch.cuda.synchronize()
-            ms = float(np.mean([a.elapsed_time(b) for a, b in ts]))
-            sweep.append({"beta": beta, "density": round(fc2["density"], 4),
-                          "density_tokens": round(fc2["density_tokens"], 4), "fwd_ms": round(ms, 4),
-                          "dense_equiv_tflops": round(dense / (ms * 1e-3) / 1e12, 1),
-                          "computed_tile_frac": round(fc2["kept"] / (ms * 1e-3) / 1e12 / PEAK_BF16, 4)})
+            sweep.append(beta_point(sol, wl, tq, tk, tv, ws, out, dens, beta, flush, stream,
+                                    max(3, args.steps // 2), dense))
 
     # ---- routing rules at matched density (threshold, per-head beta, top-k, top-p), for the record
     routes = None
-    if not args.no_route_compare:
+    if args.route_compare:
         routes = compare_routes(sol, tq, tk, tv, ws, out, dens, flush, stream, args.beta,
                                 max(3, args.steps // 2))
 
@@ -490,6 +575,13 @@ def run_ours(args, wl):
         dist.destroy_process_group()
     if rank != 0:
         return
+
+    # ---- the density >= 0.3 regime on the Wan2.1 / Hunyuan shapes (rank 0, N = 1 only)
+    dense_block = None
+    if world == 1 and not args.no_dense_block and wl.name in ("long", "wan", "hunyuan"):
+        del tq, tk, tv, out
+        torch.cuda.empty_cache()
+        dense_block = dense_regime(sol, dev, flush, stream, max(3, args.steps // 5), d)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
@@ -501,8 +593,8 @@ def run_ours(args, wl):
 
     achieved = (fc["kept"] + fc["corr"]) / (mean_fwd * 1e-3) / 1e12
     kh = kernel_hash()
-    tr = NCU_TRAFFIC.get((wl.name, wl.d, args.beta))
-    traffic = tr["bytes"] if tr and tr["kernel"] == kh else None
+    tr = NCU_TRAFFIC.get((wl.name.split("_")[0], wl.d, args.beta))
+    traffic = tr["bytes_per_head"] * B * H if tr and tr["kernel"] == kh else None
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
@@ -530,7 +622,10 @@ def run_ours(args, wl):
         "clocks": sampler.summary(),
         "workspace_bytes": sol.sol_attn_workspace_bytes(B, H, N, d),
         "kernel_sha": kh,
+        "input_gen_s": round(gen_s, 2),
     }
+    if dense_block:
+        line["density_ge_0.3"] = dense_block
     if sweep:
         line["sweep"] = sweep
     if routes:
@@ -549,24 +644,35 @@ def main():
     ap.add_argument("--shard", choices=["none", "heads"], default="none",
                     help="with N > 1: split the workload's heads over the ranks and all-gather the "
                          "outputs (strong scaling) instead of N independent replicas (weak)")
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mid", choices=sorted(inputs.WORKLOADS))
-    ap.add_argument("--beta", type=float, default=0.5)
+    ap.add_argument("--workload", default="long", choices=sorted(inputs.WORKLOADS),
+                    help="default: the long-video stress shape, the largest single-GPU workload")
+    ap.add_argument("--beta", type=float, default=None,
+                    help="routing offset (default: the first of the workload's beta sweep)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only the first this many heads of the workload (small profiling cases)")
     ap.add_argument("--sweep", action="store_true", help="also time fwd over the workload's beta sweep")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline sample time")
     ap.add_argument("--ref-seconds", type=float, default=90.0, help="target total time of the oracle arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-route-compare", action="store_true",
-                    help="skip the routing-rule comparison at matched density")
+    ap.add_argument("--no-dense-block", action="store_true",
+                    help="skip the Wan2.1/Hunyuan timings at beta 0.25 and 0 (density >= 0.3)")
+    ap.add_argument("--route-compare", action="store_true",
+                    help="also compare the routing rules at matched density (threshold, per-head "
+                         "beta, top-k, top-p)")
     ap.add_argument("--head-dim", type=int, choices=[64, 128], default=None,
                     help="generate the workload with this head dimension instead of its own")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = inputs.WORKLOADS[args.workload]
+    if args.beta is None:
+        args.beta = wl.betas[0]
     if args.head_dim is not None and args.head_dim != wl.d:
         wl = dataclasses.replace(wl, d=args.head_dim, name=f"{wl.name}_d{args.head_dim}")
+    if args.heads is not None and args.heads < wl.H:
+        wl = dataclasses.replace(wl, H=args.heads, name=f"{wl.name}_h{args.heads}")
     if args.impl == "reference":
         run_reference(args, wl)
     else:

@@ -135,19 +135,24 @@ def gen_head(seed: int, b: int, h: int, grid, d: int = HEAD_DIM, f_max: float = 
     return tuple(out)
 
 
-def gen_workload(wl: Workload, heads=None, processes: int | None = None, n_tokens: int | None = None):
+def gen_workload(wl: Workload, heads=None, processes: int | None = None, n_tokens: int | None = None,
+                 out=None):
     """All heads of a workload: q, k, v uint16 [B, H, N, d].
 
     ``heads`` restricts generation to a list of (b, h) pairs (others are left zero).
+    ``out`` = (q, k, v): caller arrays of that shape and dtype to fill instead (for example views
+    of pinned host buffers); heads not generated are left as they are.
     Heads are generated by a pool of threads (numpy releases the GIL in the random draws, the
     matrix products and the element-wise passes), each writing its own slices of the outputs;
     ``processes`` caps the thread count (default: the usable cores, at most 32).
     """
     n = wl.N if n_tokens is None else n_tokens
     shape = (wl.B, wl.H, n, wl.d)
-    q = np.zeros(shape, np.uint16)
-    k = np.zeros(shape, np.uint16)
-    v = np.zeros(shape, np.uint16)
+    if out is None:
+        q, k, v = (np.zeros(shape, np.uint16) for _ in range(3))
+    else:
+        q, k, v = out
+        assert all(a.shape == shape and a.dtype == np.uint16 for a in out)
     todo = [(b, h) for b in range(wl.B) for h in range(wl.H)] if heads is None else list(heads)
 
     def one(bh):

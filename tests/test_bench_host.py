@@ -68,3 +68,18 @@ def test_density_spread_hand_computed():
     assert abs(s["density"] - 0.5) < 1e-15
     assert abs(s["tile_density_std"] - tiles.std()) < 1e-15
     assert s["head_density_std"] == 0.0          # both heads average 0.5
+
+
+def test_mask_flop_counts_matches_flop_counts():
+    """The torch form used on full-size device masks equals the numpy definition above."""
+    rng = np.random.default_rng(3)
+    for N, BH in [(208, 1), (64 * 9, 2), (64 * 70 + 5, 3), (1, 1)]:
+        Nk = (N + 63) // 64
+        for p in (0.0, 0.3, 1.0):
+            mask = (rng.random((BH, Nk, Nk)) < p).astype(np.uint8)
+            a = bench.flop_counts(mask, N, d=128)
+            b = bench.mask_flop_counts(torch.from_numpy(mask), N, d=128)
+            for key in ("kept", "corr", "executed"):
+                assert a[key] == b[key], (N, p, key)
+            assert abs(a["density"] - b["density"]) < 1e-15
+            assert abs(a["density_tokens"] - b["density_tokens"]) < 1e-15
