@@ -42,6 +42,8 @@ FLUSH_BYTES = 256 << 20
 # keyed by (workload, head dim, beta); valid only for the kernel source whose sha256 prefix is given.
 NCU_TRAFFIC = {
     ("mid", 128, 0.5): {"bytes_per_head": (154706432 + 33871872) / 12, "kernel": "a5565cff4574a267"},
+    # two-head slice of the long-video stress shape (profiles/sol_fwd_long_beta1.5.md)
+    ("long", 128, 1.5): {"bytes_per_head": (2249162496 + 131503360) / 2, "kernel": "95b2fd9d93199bd3"},
 }
 
 
