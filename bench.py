@@ -41,9 +41,10 @@ FLUSH_BYTES = 256 << 20
 # launch over the workload's first heads (heads are independent, so traffic scales with them),
 # keyed by (workload, head dim, beta); valid only for the kernel source whose sha256 prefix is given.
 NCU_TRAFFIC = {
-    ("mid", 128, 0.5): {"bytes_per_head": (154706432 + 33871872) / 12, "kernel": "a5565cff4574a267"},
+    # full capture of one launch of the whole workload (profiles/sol_fwd_mid_beta0.5.md)
+    ("mid", 128, 0.5): {"bytes_per_head": (154629632 + 34969344) / 12, "kernel": "100d3f0f82386635"},
     # two-head slice of the long-video stress shape (profiles/sol_fwd_long_beta1.5.md)
-    ("long", 128, 1.5): {"bytes_per_head": (2249162496 + 131503360) / 2, "kernel": "95b2fd9d93199bd3"},
+    ("long", 128, 1.5): {"bytes_per_head": (2187119616 + 131701504) / 2, "kernel": "100d3f0f82386635"},
 }
 
 
