@@ -34,8 +34,9 @@
  *   - The library keeps no state between calls apart from per-device one-time set-up (kernel
  *     attributes, the SM count that sizes the split of the last wave of CTAs, the driver entry
  *     point for tensor-map encoding, and the two copy streams and the events sol_attn_fwd_host
- *     pipelines its copies with); it is thread-safe.  Calls that share a workspace must not
- *     overlap on the GPU.
+ *     pipelines its copies with) and a process-wide launch counter (it tags the workspace's
+ *     split counters, so that counters a failed call left behind never count for a later call);
+ *     it is thread-safe.  Calls that share a workspace must not overlap on the GPU.
  */
 #ifndef SOL_ATTN_H
 #define SOL_ATTN_H
@@ -84,7 +85,9 @@ sol_status sol_attn_pool(const void *k, const void *v, int B, int H, int N, int 
  * Work unit: a pair of query tiles of one head per CTA.  When the units do not fill the last wave
  * of CTAs (two per SM), the last units run as two CTAs each, every other item of the unit's work
  * list on each; the second of the two to finish merges both partial rows (their own running max
- * and sum) into the output.  The result is the same attention up to float rounding order. */
+ * and sum) into the output.  Calls with at least 2048 key blocks (N > 131008) launch the CTAs in
+ * clusters of two that split the proxy scoring's reads of the pooled keys.  The result is the
+ * same attention up to float rounding order. */
 sol_status sol_attn_fwd(const void *q, const void *k, const void *v, int B, int H, int N, int d,
                         float beta, void *workspace, void *out, int32_t *density_out,
                         void *stream);
