@@ -595,6 +595,13 @@ def run_ours(args, wl):
                "sample": desc, "seconds": round(dt, 2)}
 
     achieved = (fc["kept"] + fc["corr"]) / (mean_fwd * 1e-3) / 1e12
+    # Denominator: the measured burst bf16 peak for a kernel timed alone, the sustained one (a
+    # seconds-long GEMM loop under the power cap) when the timed region itself runs for seconds
+    timed_s = step_ms * args.steps * 1e-3
+    long_run = timed_s > 1.0
+    peak = PEAK_BF16_SUST if long_run else PEAK_BF16
+    peak_src = (f"bf16_tflops_sustained ({PEAK_SRC}): the timed region runs {timed_s:.1f} s"
+                if long_run else f"bf16_tflops ({PEAK_SRC}; burst): the timed region runs {timed_s:.2f} s")
     kh = kernel_hash()
     tr = NCU_TRAFFIC.get((wl.name.split("_")[0], wl.d, args.beta))
     traffic = tr["bytes_per_head"] * B * H if tr and tr["kernel"] == kh else None
@@ -613,10 +620,10 @@ def run_ours(args, wl):
         "computed_tile_frac_sustained": fc["kept"] / (mean_fwd * 1e-3) / 1e12 / PEAK_BF16_SUST,
         "executed_mma_tflops": fc["executed"] / (mean_fwd * 1e-3) / 1e12,
         "union_waste": 1.0 - (fc["kept"] + fc["corr"]) / fc["executed"],
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": PEAK_BF16, "unit": "TFLOP/s",
-                     "frac": achieved / PEAK_BF16, "traffic": traffic,
-                     "peak_source": f"bf16_tflops ({PEAK_SRC}; burst)", "kernel": "sol_fwd_kernel",
-                     "algorithmic_flops_per_launch": fc["kept"] + fc["corr"]},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                     "frac_of_burst": achieved / PEAK_BF16, "frac_of_sustained": achieved / PEAK_BF16_SUST,
+                     "kernel": "sol_fwd_kernel", "algorithmic_flops_per_launch": fc["kept"] + fc["corr"]},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "ms": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
