@@ -595,13 +595,7 @@ def run_ours(args, wl):
                "sample": desc, "seconds": round(dt, 2)}
 
     achieved = (fc["kept"] + fc["corr"]) / (mean_fwd * 1e-3) / 1e12
-    # Denominator: the measured burst bf16 peak for a kernel timed alone, the sustained one (a
-    # seconds-long GEMM loop under the power cap) when the timed region itself runs for seconds
-    timed_s = step_ms * args.steps * 1e-3
-    long_run = timed_s > 1.0
-    peak = PEAK_BF16_SUST if long_run else PEAK_BF16
-    peak_src = (f"bf16_tflops_sustained ({PEAK_SRC}): the timed region runs {timed_s:.1f} s"
-                if long_run else f"bf16_tflops ({PEAK_SRC}; burst): the timed region runs {timed_s:.2f} s")
+    peak, peak_src = roofline_peak(step_ms * args.steps * 1e-3)
     kh = kernel_hash()
     tr = NCU_TRAFFIC.get((wl.name.split("_")[0], wl.d, args.beta))
     traffic = tr["bytes_per_head"] * B * H if tr and tr["kernel"] == kh else None
@@ -646,6 +640,15 @@ def run_ours(args, wl):
 PEAKS, PEAK_SRC = load_peaks()
 PEAK_BF16 = float(PEAKS.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
 PEAK_BF16_SUST = float(PEAKS.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+
+
+def roofline_peak(timed_s: float):
+    """Denominator of the roofline: the measured burst bf16 peak for a kernel timed alone, the
+    sustained one (a seconds-long GEMM loop under the power cap) when the timed region itself
+    runs for more than a second.  Returns (TFLOP/s, description)."""
+    if timed_s > 1.0:
+        return PEAK_BF16_SUST, f"bf16_tflops_sustained ({PEAK_SRC}): the timed region runs {timed_s:.1f} s"
+    return PEAK_BF16, f"bf16_tflops ({PEAK_SRC}; burst): the timed region runs {timed_s:.2f} s"
 
 
 def main():

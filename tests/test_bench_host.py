@@ -83,3 +83,11 @@ def test_mask_flop_counts_matches_flop_counts():
                 assert a[key] == b[key], (N, p, key)
             assert abs(a["density"] - b["density"]) < 1e-15
             assert abs(a["density_tokens"] - b["density_tokens"]) < 1e-15
+
+
+def test_roofline_peak_follows_the_timed_region_length():
+    burst, src = bench.roofline_peak(0.05)            # e.g. 20 steps of 2.5 ms
+    assert burst == bench.PEAK_BF16 and "burst" in src
+    sust, src = bench.roofline_peak(3.2)              # e.g. 30 steps of 107 ms
+    assert sust == bench.PEAK_BF16_SUST and "sustained" in src
+    assert sust < burst
