@@ -238,9 +238,15 @@ sol_status route_arg(int route, double param, RouteArg *ra)
 
 // Copy streams and events of the pipelined host entry point: one set per device, created on first
 // use and kept until the process exits.  A call uses about one head group per kHostGroupBytes of
-// upload, at most kHostGroups: measured on B200 (host link ~55 GB/s each way), 12 heads x 16384
-// tokens (151 MB up) ran best with 5 groups, 24 x 118800 and 40 x 75600 (2.2-2.3 GB) with 8.
-constexpr int kHostGroups = 8;
+// upload, at most kHostGroups when a head's tile pairs leave their last wave of CTAs at least 90 %
+// full, else at most kHostGroupsRagged: each group's launch ends in that partly empty wave, which a
+// compute-bound call pays once per group.  Measured on B200 (host link ~55 GB/s each way, ~71 GB/s
+// both ways at once; with 8 / 16 / 32 groups): 32 heads x 262144 tokens (6.4 GB up, 2048 tile
+// pairs per head = 6.92 waves of 296 CTAs) 140.5 / 131.5 / 130.0 ms; 40 x 75600 (591 pairs,
+// 2.00 waves) 50.1 / 48.2 / 47.7; 24 x 118800 (929 pairs, 3.14 waves) 58.0 / 58.8 / 61.7; 12 x 16384
+// (151 MB up) ran best with 5 groups.
+constexpr int kHostGroups = 32;
+constexpr int kHostGroupsRagged = 8;
 constexpr size_t kHostGroupBytes = 32u << 20;
 
 struct HostPipe {
@@ -251,6 +257,7 @@ struct HostPipe {
     cudaEvent_t start = nullptr, done = nullptr;
     cudaEvent_t uploaded[kHostGroups] = {};
     cudaEvent_t computed[kHostGroups] = {};
+    int slots = 0;          // CTAs of the fused kernel resident at once (two per SM)
 };
 
 HostPipe g_host_pipes[64];
@@ -260,7 +267,7 @@ HostPipe *host_pipe()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     HostPipe &hp = g_host_pipes[dev];
-    std::call_once(hp.once, [&hp] {
+    std::call_once(hp.once, [&hp, dev] {
         auto event = [&hp](cudaEvent_t *e) {
             if (hp.err == cudaSuccess) hp.err = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
         };
@@ -272,6 +279,9 @@ HostPipe *host_pipe()
             event(&hp.uploaded[g]);
             event(&hp.computed[g]);
         }
+        int sms = 0;
+        if (hp.err == cudaSuccess) hp.err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        hp.slots = 2 * sms;
     });
     return hp.err == cudaSuccess ? &hp : nullptr;
 }
@@ -436,8 +446,11 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
     // compute.  The last download is joined back into `stream`.
     const size_t head_bytes = static_cast<size_t>(s.N) * static_cast<size_t>(s.d) * 2;
     const size_t upload = 3 * head_bytes * static_cast<size_t>(s.BH);
+    const long long slots = std::max(1, hp->slots);
+    const long long last_wave = ((s.Nq + 1) / 2) % slots;   // a head's tile pairs in its last wave
+    const bool full_waves = last_wave == 0 || 10 * last_wave >= 9 * slots;
     const int G = static_cast<int>(std::min<size_t>(
-        std::min<size_t>(kHostGroups, static_cast<size_t>(s.BH)),
+        std::min<size_t>(full_waves ? kHostGroups : kHostGroupsRagged, static_cast<size_t>(s.BH)),
         std::max<size_t>(1, (upload + kHostGroupBytes - 1) / kHostGroupBytes)));
     const size_t head_dens = static_cast<size_t>(s.Nq) * sizeof(int32_t);
     auto fail = [](cudaError_t e) { return e != cudaSuccess; };

@@ -175,8 +175,9 @@ sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream);
 
 /* One end-to-end call on host buffers: copies q, k, v from (preferably pinned) host memory into
  * the caller's device buffers, pools, runs the forward, and copies out and density back, without
- * synchronising.  The heads are split into up to 8 contiguous groups (about one per 32 MiB of
- * upload; the first and the last group half the size of the others) and the copies are pipelined
+ * synchronising.  The heads are split into contiguous groups (about one per 32 MiB of upload, at
+ * most 32 when one head's tile pairs fill their last wave of CTAs at least 90 %, else at most 8;
+ * the first and the last group half the size of the others) and the copies are pipelined
  * with the compute: group g+1 uploads on an internal copy stream while `stream` pools and runs
  * group g, and group g's output downloads on a second internal copy stream while later groups
  * compute.  The uploads wait for all work queued on `stream` before this call, and everything
