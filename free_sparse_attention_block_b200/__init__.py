@@ -242,6 +242,8 @@ def sol_attn_fwd_debug(q, k, v, beta: float, workspace, out, density_out=None, p
 
 
 def sol_attn_read_status(workspace, stream=None):
+    """Synchronise the stream, read and clear the device status words: (status code, wait site).
+    workspace None reads the status of sol_attn_fwd_noalloc's built-in scratch on this device."""
     where = C.c_int(0)
     st = load_library().sol_attn_read_status(_ptr(workspace), C.byref(where), _stream(stream))
     return st, where.value
