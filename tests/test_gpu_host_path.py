@@ -50,11 +50,14 @@ class HostCall:
 
 
 @pytest.mark.parametrize("B,H,N,d", [(1, 1, 1000, 128), (1, 3, 64 * 9 + 16, 128), (2, 7, 4096 + 5, 128),
-                                     (1, 12, 4096, 64), (1, 9, 2048, 128), (1, 12, 4096, 128)])
+                                     (1, 12, 4096, 64), (1, 9, 2048, 128), (1, 12, 4096, 128),
+                                     (1, 12, 37888, 128)])
 def test_host_path_matches_device_path(B, H, N, d):
     """(1, 12, 4096, 128) uploads 37.7 MB, so the host path runs two head groups, and its 384
     work units leave a last wave of 88 of 296 CTAs, so the call splits its last 128 units: each
-    group launch must split exactly the call's units among its own."""
+    group launch must split exactly the call's units among its own.  (1, 12, 37888, 128) uploads
+    349 MB with 296 tile pairs per head, which fill their last wave of CTAs on a 148-SM part, so
+    the host path runs 11 head groups (the rule that allows more than 8)."""
     q, k, v = inputs.small_workload(N, BH=B * H, seed=N + d, d=d)
     q, k, v = (x.reshape(B, H, N, d) for x in (q, k, v))
     ref_out, ref_dens = device_reference(q, k, v, 0.7)
