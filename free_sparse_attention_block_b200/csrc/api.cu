@@ -458,6 +458,14 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
         fail(cudaEventRecord(hp->start, cs)) || fail(cudaStreamWaitEvent(hp->up, hp->start, 0)) ||
         fail(cudaStreamWaitEvent(hp->down, hp->start, 0)))
         return SOL_ERR_CUDA;
+    // An error return after this point still orders the copies already queued on the internal
+    // streams before later work on `stream` (best effort: the joins themselves may fail too), so
+    // that the caller's buffers are not read or written behind its back.
+    auto join_and = [&](sol_status status) {
+        if (cudaEventRecord(hp->done, hp->down) == cudaSuccess) cudaStreamWaitEvent(cs, hp->done, 0);
+        if (cudaEventRecord(hp->start, hp->up) == cudaSuccess) cudaStreamWaitEvent(cs, hp->start, 0);
+        return status;
+    };
     // group g covers heads [edge(g), edge(g+1)); the first and the last group get half the weight
     // of the others: the first one's upload delays the compute of a compute-bound call, the last
     // one's compute and download follow the last upload of a link-bound one
@@ -481,7 +489,7 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
             fail(cudaMemcpyAsync(gk, static_cast<const uint8_t *>(h_k) + off, bytes, cudaMemcpyHostToDevice, hp->up)) ||
             fail(cudaMemcpyAsync(gv, static_cast<const uint8_t *>(h_v) + off, bytes, cudaMemcpyHostToDevice, hp->up)) ||
             fail(cudaEventRecord(hp->uploaded[g], hp->up)) || fail(cudaStreamWaitEvent(cs, hp->uploaded[g], 0)))
-            return SOL_ERR_CUDA;
+            return join_and(SOL_ERR_CUDA);
         Shape gs = s;
         gs.BH = h1 - h0;
         const Pooled pw = pooled_at(workspace, s, h0);
@@ -490,17 +498,17 @@ sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, 
         if (st == SOL_OK)
             st = launch_fwd(gq, gk, gv, gs, pw, beta, nullptr, go, gd, nullptr, nullptr, nullptr, 0,
                             kDefaultTimeoutNs, cs, RouteArg{});
-        if (st != SOL_OK) return st;
+        if (st != SOL_OK) return join_and(st);
         if (fail(cudaEventRecord(hp->computed[g], cs)) || fail(cudaStreamWaitEvent(hp->down, hp->computed[g], 0)) ||
             fail(cudaMemcpyAsync(static_cast<uint8_t *>(h_out) + off, go, bytes, cudaMemcpyDeviceToHost, hp->down)))
-            return SOL_ERR_CUDA;
+            return join_and(SOL_ERR_CUDA);
         if (h_density &&
             fail(cudaMemcpyAsync(h_density + static_cast<size_t>(h0) * s.Nq, gd,
                                  static_cast<size_t>(h1 - h0) * head_dens, cudaMemcpyDeviceToHost, hp->down)))
-            return SOL_ERR_CUDA;
+            return join_and(SOL_ERR_CUDA);
     }
     if (fail(cudaEventRecord(hp->done, hp->down)) || fail(cudaStreamWaitEvent(cs, hp->done, 0)))
-        return SOL_ERR_CUDA;
+        return join_and(SOL_ERR_CUDA);
     return SOL_OK;
 }
 

@@ -183,8 +183,10 @@ sol_status sol_attn_read_status(void *workspace, int *where_out, void *stream);
  * compute.  The uploads wait for all work queued on `stream` before this call, and everything
  * (the last download included) is ordered before work queued on `stream` after it, so the device
  * buffers may be reused by the next call.  Host buffers must stay valid until `stream` reaches
- * that point.  h_density / d_density may both be NULL.  workspace: 256-byte aligned, as for
- * sol_attn_pool.  Results are bit-identical to sol_attn_pool + sol_attn_fwd. */
+ * that point.  An error returned after copies were queued keeps that ordering (as far as the
+ * failing CUDA runtime allows), so the same rule applies.  h_density / d_density may both be NULL.
+ * workspace: 256-byte aligned, as for sol_attn_pool.  Results are bit-identical to sol_attn_pool +
+ * sol_attn_fwd. */
 sol_status sol_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, int B, int H,
                              int N, int d, float beta, void *d_q, void *d_k, void *d_v,
                              void *workspace, void *d_out, int32_t *d_density, void *h_out,
