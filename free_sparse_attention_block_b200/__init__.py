@@ -293,15 +293,32 @@ def workspace_views(workspace, B: int, H: int, N: int, d: int = HEAD_DIM):
     return k32, v32, k16, v16
 
 
+def _torch_stream(stream, device):
+    """`stream` (a torch stream or a raw cudaStream_t handle) as a torch stream object."""
+    import torch
+    if isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream), device=device)
+
+
 def forward(q, k, v, beta: float, stream=None):
     """Pool + fused forward on device tensors.  Allocates the workspace, output and density with
     torch (the library itself allocates nothing).  Returns (out bf16 [B,H,N,d], density int32
-    [B,H,Nq])."""
+    [B,H,Nq]).  With a `stream` other than the current one, the kernels run on it after the work
+    already queued on the current stream; the results are ready when that stream reaches them
+    (the caller synchronises before using them elsewhere), and the caching allocator keeps the
+    workspace, freed on return, until the stream's kernels are done."""
     import torch
     B, H, N, d = _shape(q)
     ws = torch.empty(sol_attn_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
     out = torch.empty_like(q)
     dens = torch.empty((B, H, (N + TILE - 1) // TILE), dtype=torch.int32, device=q.device)
+    if stream is not None:
+        s = _torch_stream(stream, q.device)
+        if s != torch.cuda.current_stream(q.device):
+            s.wait_stream(torch.cuda.current_stream(q.device))
+            for t in (ws, out, dens):
+                t.record_stream(s)
     sol_attn_pool(k, v, ws, stream)
     sol_attn_fwd(q, k, v, beta, ws, out, dens, stream)
     return out, dens

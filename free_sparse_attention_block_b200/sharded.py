@@ -71,4 +71,11 @@ def sol_attn_fwd_sharded(q, k, v, beta: float, H: int, group=None, gather: bool 
     out, dens = forward(q, k, v, beta, stream)
     if not gather:
         return out, dens
+    if stream is not None and q.is_cuda:
+        # the collective is ordered after the current stream's work, so that stream waits for
+        # the forward's
+        import torch
+
+        from . import _torch_stream
+        torch.cuda.current_stream(q.device).wait_stream(_torch_stream(stream, q.device))
     return gather_heads(out, H, group), gather_heads(dens, H, group)

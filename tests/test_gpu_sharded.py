@@ -40,6 +40,11 @@ def test_one_rank_nccl_group_against_the_oracle():
         ref = gpu_run(q, k, v, 0.7)           # the GPU's masks and statistics (debug outputs)
         g = dict(ref, out=got_out.float().cpu().numpy(), density=got_dens.cpu().numpy())
         check_parity(q, k, v, 0.7, g, default_units(H, (N + 63) // 64, None))
+        side = torch.cuda.Stream()     # the gather must wait for a forward queued on another stream
+        got_out, got_dens = sol_attn_fwd_sharded(tq, tk, tv, 0.7, H, stream=side)
+        torch.cuda.synchronize()
+        assert torch.equal(got_out.view(torch.int16), want_out.view(torch.int16))
+        assert torch.equal(got_dens, want_dens)
         with pytest.raises(ValueError):
             sol_attn_fwd_sharded(tq[:, :4], tk[:, :4], tv[:, :4], 0.7, H)   # not this rank's heads
     finally:
